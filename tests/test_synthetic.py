@@ -1,0 +1,55 @@
+"""The seeded input generator (no GPU)."""
+import numpy as np
+import torch
+
+from adaptive_vector_quantized_avq_b200 import synthetic as syn
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(100000) * 10.0 ** rng.integers(-6, 6, 100000),
+                        [0.0, -0.0, 1.0, 3.75, -4.0, 1e-30]])
+    ours = syn.f64_to_bf16_bits(x)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    back = syn.bf16_bits_to_f64(ours)
+    assert np.array_equal(back, torch.from_numpy(ours.view(np.int16)).view(torch.bfloat16).double().numpy())
+
+
+def test_codebook_constraint_exact_in_storage_dtype():
+    for name in ("tiny-fp32", "vit-b", "refine-d128"):
+        wl = syn.WORKLOADS[name].with_(B=1, N=8)
+        inp = syn.generate(wl)
+        cb = inp.f64("codebook")
+        assert cb.shape == (wl.H, wl.Mtot, wl.d)
+        par = cb[:, :wl.M0]
+        kids = cb[:, wl.M0:].reshape(wl.H, wl.M0, wl.C, wl.d)
+        assert np.array_equal(par * wl.C, kids.sum(axis=2))
+        # values are on the 2^-5 grid and survive the storage round trip
+        assert np.array_equal(np.rint(cb / syn.GRID) * syn.GRID, cb)
+        assert np.array_equal(syn.storage_to_f64(syn.to_storage(cb, wl.dtype), wl.dtype), cb)
+
+
+def test_generator_is_deterministic_and_seeded():
+    wl = syn.small_workload(N=64, d=8, M0=4, C=2, dtype="bf16", B=2, H=3)
+    a, b = syn.generate(wl), syn.generate(wl)
+    for k in ("K", "V", "Q", "codebook"):
+        assert np.array_equal(getattr(a, k), getattr(b, k))
+    c = syn.generate(wl.with_(seed=1))
+    assert not np.array_equal(a.K, c.K)
+    assert a.K.dtype == np.uint16 and a.K.shape == (2, 3, 64, 8)
+
+
+def test_mixture_statistics():
+    wl = syn.small_workload(N=20000, d=16, M0=8, C=2, n_components=8, sigma=0.3, seed=3)
+    inp = syn.generate(wl)
+    K = inp.f64("K")[0, 0]
+    cb = inp.f64("codebook")[0, :8]
+    d2 = ((K[:, None, :] - cb[None]) ** 2).sum(-1).min(1)
+    # nearest-centre squared distance ~ d*sigma^2 (+ small child-mean offset)
+    assert 0.8 * 16 * 0.09 < np.median(d2) < 1.6 * 16 * 0.09
+
+
+def test_zipf_weights_heavy_first():
+    w = syn._mixture_weights(256, 1.1)
+    assert np.all(np.diff(w) < 0) and abs(w.sum() - 1) < 1e-12
