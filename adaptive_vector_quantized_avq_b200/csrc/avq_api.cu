@@ -1,0 +1,143 @@
+// avq_api.cu -- the extern "C" entry points declared in include/avq.h:
+// argument validation on the host, zeroing of outputs on the stream, and the
+// choice of kernel for the shape and dtype.
+#include <stdint.h>
+
+#include <atomic>
+
+#include "avq_internal.cuh"
+
+namespace avq {
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace avq
+
+namespace avq {
+cudaError_t launch_precompute_simt(const avq_shape& s, const void* K, const void* V,
+                                   const void* cb, int32_t* assign, int32_t* counts,
+                                   float* vsum, cudaStream_t st);
+cudaError_t launch_attention_simt(const avq_shape& s, const void* Q, const void* cb,
+                                  const int32_t* counts, const float* vsum, int P, int tile,
+                                  float scale, void* O, int32_t* selected, cudaStream_t st);
+size_t attention_simt_smem(const avq_shape& s);
+}  // namespace avq
+
+using namespace avq;
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_shape(const avq_shape* s) {
+    if (!s) return AVQ_EINVAL;
+    if (s->B < 1 || s->H < 1 || s->N < 0) return AVQ_EINVAL;
+    if (s->d != 64 && s->d != 128) return AVQ_EINVAL;
+    if (s->dtype != AVQ_F32 && s->dtype != AVQ_BF16) return AVQ_EINVAL;
+    if (s->M0 < 1 || s->C < 1) return AVQ_EINVAL;
+    if (s->M0 > kMaxM0 || s->C > kMaxC) return AVQ_EUNSUPPORTED;
+    // element counts must fit the kernels' index arithmetic
+    const long long rows = (long long)s->B * s->H * s->N;
+    if (rows * s->d >= (1LL << 40)) return AVQ_EUNSUPPORTED;
+    if ((long long)s->B * s->H > 65535LL * 32) return AVQ_EUNSUPPORTED;
+    return AVQ_OK;
+}
+
+int check_ws(const void* ws, size_t have, size_t need) {
+    if (need == 0) return AVQ_OK;
+    if (!ws || have < need) return AVQ_EWORKSPACE;
+    if (!aligned(ws, 256)) return AVQ_EINVAL;
+    return AVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int avq_version(void) { return 100; }
+
+uint64_t avq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* avq_status_string(int st) {
+    switch (st) {
+        case AVQ_OK: return "AVQ_OK";
+        case AVQ_EINVAL: return "AVQ_EINVAL: invalid argument (null or misaligned pointer, size out of range)";
+        case AVQ_EUNSUPPORTED: return "AVQ_EUNSUPPORTED: sizes beyond the on-chip limits of the kernels";
+        case AVQ_ECUDA: return "AVQ_ECUDA: a CUDA call failed";
+        case AVQ_ETIMEOUT: return "AVQ_ETIMEOUT: a bounded device-side wait ran out";
+        case AVQ_EWORKSPACE: return "AVQ_EWORKSPACE: workspace missing or too small";
+        default: return "unknown avq status";
+    }
+}
+
+size_t avq_precompute_workspace_bytes(const avq_shape* s) {
+    if (check_shape(s) != AVQ_OK) return 0;
+    return kStatusBytes;
+}
+
+int avq_precompute(const avq_shape* s, const void* K, const void* V, const void* codebook,
+                   int32_t* assign, int32_t* counts, float* vsum, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc != AVQ_OK) return rc;
+    if (!codebook || !counts || !vsum) return AVQ_EINVAL;
+    if (s->N > 0 && (!K || !V || !assign)) return AVQ_EINVAL;
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(codebook, 16) || !aligned(vsum, 16) ||
+        !aligned(assign, 4) || !aligned(counts, 4))
+        return AVQ_EINVAL;
+    rc = check_ws(workspace, workspace_bytes, avq_precompute_workspace_bytes(s));
+    if (rc != AVQ_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t Mtot = (size_t)s->M0 * (1 + s->C);
+    const size_t BH = (size_t)s->B * s->H;
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * BH * Mtot, st) != cudaSuccess) return AVQ_ECUDA;
+    if (cudaMemsetAsync(vsum, 0, sizeof(float) * BH * Mtot * s->d, st) != cudaSuccess) return AVQ_ECUDA;
+    if (s->N == 0) return AVQ_OK;
+    cudaError_t e = launch_precompute_simt(*s, K, V, codebook, assign, counts, vsum, st);
+    return e == cudaSuccess ? AVQ_OK : AVQ_ECUDA;
+}
+
+size_t avq_attention_workspace_bytes(const avq_shape* s, int P, int tile) {
+    if (check_shape(s) != AVQ_OK) return 0;
+    if (P < 0 || P > s->M0 || (tile != 64 && tile != 128)) return 0;
+    return kStatusBytes;
+}
+
+int avq_attention(const avq_shape* s, const void* Q, const void* codebook, const int32_t* counts,
+                  const float* vsum, int P, int tile, float scale, void* O, int32_t* selected,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_shape(s);
+    if (rc != AVQ_OK) return rc;
+    if (P < 0 || P > s->M0 || (tile != 64 && tile != 128)) return AVQ_EINVAL;
+    if (!(scale > 0.f) || !(scale < 3.0e38f)) return AVQ_EINVAL;
+    if (!codebook || !counts || !vsum) return AVQ_EINVAL;
+    if (s->N > 0 && (!Q || !O || (P > 0 && !selected))) return AVQ_EINVAL;
+    if (!aligned(Q, 16) || !aligned(O, 16) || !aligned(codebook, 16) || !aligned(vsum, 16) ||
+        !aligned(counts, 4) || !aligned(selected, 4))
+        return AVQ_EINVAL;
+    rc = check_ws(workspace, workspace_bytes, avq_attention_workspace_bytes(s, P, tile));
+    if (rc != AVQ_OK) return rc;
+    if (s->N == 0) return AVQ_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_attention_simt(*s, Q, codebook, counts, vsum, P, tile, scale, O,
+                                          selected, st);
+    return e == cudaSuccess ? AVQ_OK : AVQ_ECUDA;
+}
+
+int avq_device_status(void* workspace, void* stream) {
+    if (!workspace || !aligned(workspace, 256)) return AVQ_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    StatusBlock host;
+    if (cudaMemcpyAsync(&host, workspace, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return AVQ_ECUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return AVQ_ECUDA;
+    if (host.error != 0) {
+        const int32_t zero = 0;
+        if (cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return AVQ_ECUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return AVQ_ECUDA;
+        return host.error;
+    }
+    return AVQ_OK;
+}
+
+}  // extern "C"

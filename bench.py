@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Throughput of the AVQ-attention forward path on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+``avq_precompute`` (assignment + full-tree statistics) then ``avq_attention``
+(parent attention, importance, top-P, child correction, output), through the
+C ABI. Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--P P]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+Multi-GPU (N > 1, launched by torch.distributed.run): every rank runs the
+same workload on its own seeded batch (heads are independent, no data-path
+collective): weak scaling, value = all ranks' query rows / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from adaptive_vector_quantized_avq_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "AVQ forward queries/sec and % of roofline (HBM/tensor) at N=64k, 1×B200"
+UNIT = "queries/s"
+DEFAULT_WORKLOAD = "max-64k"
+L2_BYTES = 126 * 2 ** 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def algorithmic(wl: syn.Workload, P: int):
+    """Per-call algorithmic bytes and tensor FLOPs (paper Table 1 cost model):
+    precompute reads K and V and evaluates M0 + C distances per key;
+    attention reads Q, writes O and evaluates M0 + P*C logits and weighted
+    sums per query."""
+    s = 2 if wl.dtype == "bf16" else 4
+    R, d = wl.rows, wl.d
+    return {
+        "precompute": {"bytes": 2 * R * d * s, "flops": 2 * R * (wl.M0 + wl.C) * d},
+        "attention": {"bytes": 2 * R * d * s, "flops": 4 * R * (wl.M0 + P * wl.C) * d},
+    }
+
+
+def roofline_for(kind, alg, ms, peaks, sustained):
+    hbm = peaks["hbm_gbs"]
+    tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    t_hbm = alg["bytes"] / (hbm * 1e9)
+    t_ten = alg["flops"] / (tf * 1e12)
+    sec = ms / 1e3
+    if t_ten > t_hbm:
+        ach = alg["flops"] / sec / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": tf, "unit": "TFLOP/s", "frac": ach / tf,
+                "roofline_us": t_ten * 1e6}
+    ach = alg["bytes"] / sec / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+            "roofline_us": t_hbm * 1e6}
+
+
+def kernel_source_hash(kind: str) -> str:
+    """Hash of the sources a kernel is built from (to invalidate stored ncu traffic)."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "adaptive_vector_quantized_avq_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kind: str, workload: str, P: int):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel sources
+    are unchanged since it was taken; else None."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    with open(PROFILE_TRAFFIC) as f:
+        d = json.load(f)
+    e = d.get(f"{kind}/{workload}/P{P}")
+    if not e or e.get("source_hash") != kernel_source_hash(kind):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the GPU works."""
+
+    Q = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+         "utilization.gpu")
+
+    def __init__(self, bus_id: str | None, period_ms: int = 50):
+        self.bus_id = bus_id
+        self.period_ms = period_ms
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                   f"-lms={self.period_ms}", f"--filename={self.path}"]
+            if self.bus_id:
+                cmd.insert(1, f"--id={self.bus_id}")
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(self.period_ms / 1000 * 2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 11:
+                    continue
+                try:
+                    rows.append({"sm": float(p[2]), "max": float(p[3]), "power": float(p[4]),
+                                 "hw": p[6], "hwt": p[7], "swt": p[8], "pcap": p[9],
+                                 "util": float(p[10])})
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        busy = [r for r in rows if r["util"] > 0] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(busy), "power_w_max": max(r["power"] for r in busy)}
+
+
+def bus_id_of(torch, dev: int) -> str | None:
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------- CPU oracle timing
+class OracleSampler:
+    """The fp64 oracle timed on a bounded sample of the workload: the first
+    ``n`` keys of head (0,0) through the precompute and the first ``n`` query
+    rows (whole tiles) through the attention, using that head's full
+    statistics (computed once, untimed, like inputs already resident)."""
+
+    def __init__(self, wl: syn.Workload, P: int):
+        from oracle import oracle as orc
+        self.O = orc.get()
+        self.threads = self.O.max_threads()
+        self.wl, self.P = wl, P
+        one = wl.with_(B=1, H=1)
+        inp = syn.generate(one)
+        self.K, self.V, self.Q, self.cb = (inp.f64(n) for n in ("K", "V", "Q", "codebook"))
+        self.full = self.O.precompute(self.K, self.V, self.cb, wl.M0, wl.C, nthreads=self.threads)
+        self.ntiles = one.ntiles
+
+    def run(self, n_tiles: int):
+        wl = self.wl
+        n_tiles = max(1, min(self.ntiles, n_tiles))
+        n = min(wl.N, n_tiles * wl.tile)
+        t0 = time.perf_counter()
+        self.O.precompute(self.K[:, :, :n], self.V[:, :, :n], self.cb, wl.M0, wl.C,
+                          nthreads=self.threads)
+        self.O.attention(self.Q, self.cb, self.full["counts"], self.full["vsum"], wl.M0, wl.C,
+                         self.P, wl.tile, wl.softmax_scale, tile_ids=np.arange(n_tiles),
+                         nthreads=self.threads)
+        return n, time.perf_counter() - t0
+
+    def tiles_for(self, seconds: float) -> int:
+        n, dt = self.run(2)
+        per_row = dt / n
+        return int(max(1, min(self.ntiles, math.ceil(seconds / per_row / self.wl.tile))))
+
+    def describe(self, n_tiles: int) -> str:
+        n = min(self.wl.N, n_tiles * self.wl.tile)
+        return (f"{n} keys precomputed + {n} queries attended ({n_tiles} tiles of "
+                f"{self.wl.tile}) of head (0,0) of {self.wl.name}; fp64 oracle, "
+                f"{self.threads} OpenMP threads")
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from adaptive_vector_quantized_avq_b200 import binding as bd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    wl = syn.WORKLOADS[args.workload]
+    P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
+    wl_rank = wl.with_(seed=wl.seed + rank)
+    inp = syn.generate(wl_rank)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+    def to_dev(a):
+        if wl.dtype == "bf16":
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    def pinned(a):
+        t = torch.from_numpy(a.view(np.int16) if wl.dtype == "bf16" else a)
+        return t.pin_memory()
+
+    K, V, Q, cb = (to_dev(getattr(inp, n)) for n in ("K", "V", "Q", "codebook"))
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    Mtot = wl.Mtot
+    shape = bd.make_shape(B, H, N, d, wl.M0, wl.C, tdt)
+    assign = torch.empty((B, H, N), dtype=torch.int32, device=dev)
+    counts = torch.empty((B, H, Mtot), dtype=torch.int32, device=dev)
+    vsum = torch.empty((B, H, Mtot, d), dtype=torch.float32, device=dev)
+    O = torch.empty_like(Q)
+    sel = torch.empty((B, H, wl.ntiles, max(P, 1)), dtype=torch.int32, device=dev)
+    ws_pre = bd.workspace(bd.avq_precompute_workspace_bytes(shape), dev)
+    ws_att = bd.workspace(bd.avq_attention_workspace_bytes(shape, P, wl.tile), dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    scale = wl.softmax_scale
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rc = bd.avq_precompute(shape, K, V, cb, assign, counts, vsum, ws_pre, ws_pre.numel(), sp)
+        if ev is not None:
+            ev[1].record(stream)
+        rc2 = bd.avq_attention(shape, Q, cb, counts, vsum, P, wl.tile, scale, O,
+                               sel if P > 0 else None, ws_att, ws_att.numel(), sp)
+        if ev is not None:
+            ev[2].record(stream)
+        if rc or rc2:
+            raise RuntimeError(f"avq call failed: {rc} {rc2}")
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if bd.avq_device_status(ws_pre, sp) or bd.avq_device_status(ws_att, sp):
+        raise RuntimeError("device status error after warm-up")
+
+    clocks = ClockSampler(bus_id_of(torch, local))
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = bd.avq_kernel_launches()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = bd.avq_kernel_launches() - launches0
+    barrier()
+    clk = clocks.stop()
+    ms_total = start.elapsed_time(stop)
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    att_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if bd.avq_device_status(ws_pre, sp) or bd.avq_device_status(ws_att, sp):
+        raise RuntimeError("device status error after timing")
+
+    # end to end through the public API: pinned host inputs in, output out
+    hK, hV, hQ, hcb = (pinned(getattr(inp, n)) for n in ("K", "V", "Q", "codebook"))
+    hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for h_, d_ in ((hK, K), (hV, V), (hQ, Q), (hcb, cb)):
+            d_.view(h_.dtype).copy_(h_, non_blocking=True)
+        step()
+        hO.copy_(O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    barrier()
+    h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ, hcb))
+    d2h = hO.numel() * hO.element_size()
+
+    # max over ranks
+    vals = torch.tensor([ms_total, e2e_ms, statistics.mean(pre_ms), statistics.mean(att_ms)],
+                        device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms, pre_avg, att_avg = vals.tolist()
+    ms_step = ms_total / args.steps
+    rows_all = wl.rows * world
+    value = rows_all / (ms_step / 1e3)
+
+    out = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        alg = algorithmic(wl, P)
+        kern = {"precompute": pre_avg, "attention": att_avg}
+        dom = max(kern, key=kern.get)
+        rl = {k: roofline_for(k, alg[k], kern[k], peaks, sustained=True) for k in kern}
+        roof = dict(rl[dom])
+        roof["kernel"] = dom
+        roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if roof['bound'] == 'tensor' else 'hbm_gbs'})"
+        roof["traffic"] = stored_traffic(dom, wl.name, P)
+        roof["algorithmic_per_launch"] = alg[dom]["bytes"] if roof["bound"] == "hbm" else alg[dom]["flops"]
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "B": B, "H": H, "N": N, "d": d, "M0": wl.M0,
+                       "C": wl.C, "P": P, "tile": wl.tile, "scale": scale,
+                       "query_rows_per_gpu": wl.rows,
+                       "l2": f"no flush: Q+K+V = {3 * wl.rows * d * (2 if wl.dtype == 'bf16' else 4) / 1e6:.0f} MB "
+                             f"per step > {L2_BYTES / 1e6:.0f} MB L2",
+                       "seed": f"{wl.seed}+rank"},
+            "kernels": {k: {"ms_avg": kern[k], "ms_min": min(pre_ms if k == 'precompute' else att_ms),
+                            "roofline": rl[k]} for k in kern},
+            "roofline": roof,
+            "clocks": clk,
+            "e2e": {"value": rows_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+            "gpu_launches": int(launches),
+        }
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSampler(wl, P)
+        nt = smp.tiles_for(args.cpu_budget)
+        n, secs = smp.run(nt)
+        out["cpu_baseline"] = {"value": n / secs, "unit": UNIT, "cores": smp.threads,
+                               "kind": "oracle", "sample": smp.describe(nt), "seconds": secs}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# --------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = syn.WORKLOADS[args.workload]
+    P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
+    smp = OracleSampler(wl, P)
+    per_step = 150.0 / max(1, args.steps + args.warmup)
+    nt = smp.tiles_for(per_step)          # calibration, untimed
+    for _ in range(args.warmup):
+        smp.run(nt)
+    times = []
+    for _ in range(args.steps):
+        n, dt = smp.run(nt)
+        times.append(dt)
+    rows = n
+    cores, desc = smp.threads, smp.describe(nt)
+    ms = 1e3 * statistics.mean(times)
+    value = rows / (ms / 1e3)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "M0": wl.M0,
+                   "C": wl.C, "P": P, "tile": wl.tile, "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--P", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

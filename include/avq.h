@@ -1,0 +1,165 @@
+/*
+ * avq.h -- C ABI of the AVQ-attention forward path on NVIDIA B200 (sm_100a).
+ *
+ * AVQ-attention ("AVQ-Attention: Adaptive Vector-Quantized Attention")
+ * replaces the keys of softmax attention by codewords of a frozen two-level
+ * tree codebook and refines, per query tile, the most attended parents with
+ * their children. The forward pass is two calls:
+ *
+ *   avq_precompute  -- paper §4.2 ("Vector Quantization for (A)VQ-Attention");
+ *                      papernotes summary, Key Designs 2 (fused full-tree
+ *                      precomputation): key assignment and per-codeword
+ *                      counts and value sums for the whole tree.
+ *   avq_attention   -- paper §4.3 ("Computing (A)VQ-Attention with Flash
+ *                      Attention"); papernotes summary, Key Designs 3:
+ *                      parent attention, codeword importance, top-P parent
+ *                      selection per query tile, child attention with the
+ *                      parent-contribution correction, output.
+ *
+ * Conventions common to every call
+ * --------------------------------
+ * - Pointers named "device" must point to memory of the current CUDA device;
+ *   the caller owns and allocates every buffer. The library allocates no
+ *   memory and never synchronises the stream: each call only enqueues work
+ *   on `stream` (a cudaStream_t passed as void*; NULL is the legacy default
+ *   stream) and returns.
+ * - Tensors are dense, row-major, C-contiguous:
+ *     K, V, Q, O : [B, H, N, d]            element type `dtype`
+ *     codebook   : [H, Mtot, d]            element type `dtype`, Mtot = M0*(1+C)
+ *                  tree order: parents 0..M0-1, then child c of parent p at
+ *                  row M0 + p*C + c (each parent's children are contiguous,
+ *                  paper §4.3 "Child spawning"); one codebook per head,
+ *                  shared by the batch (paper §4.1).
+ *     assign     : [B, H, N]        int32  leaf id of each key, in tree order
+ *     counts     : [B, H, Mtot]     int32
+ *     vsum       : [B, H, Mtot, d]  float32
+ *     selected   : [B, H, ceil(N/tile), P] int32
+ * - Alignment: K, V, Q, O, codebook, vsum and the workspace 16 bytes;
+ *   assign, counts, selected 4 bytes.
+ * - Return value: AVQ_OK (0) or a negative avq_status. Argument errors are
+ *   detected on the host before anything is enqueued, and leave every output
+ *   untouched. A launch failure returns AVQ_ECUDA.
+ */
+#ifndef AVQ_B200_H
+#define AVQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of K, V, Q, O and the codebook (all the same). */
+typedef enum { AVQ_F32 = 0, AVQ_BF16 = 1 } avq_dtype;
+
+/* Problem sizes. Supported: B, H >= 1; N >= 0; d in {64, 128};
+ * 1 <= M0 <= 128; 1 <= C <= 16. */
+typedef struct {
+    int32_t B, H, N, d;
+    int32_t M0, C;
+    int32_t dtype; /* avq_dtype */
+} avq_shape;
+
+typedef enum {
+    AVQ_OK = 0,
+    AVQ_EINVAL = -1,        /* null/misaligned pointer, size or argument out of range */
+    AVQ_EUNSUPPORTED = -2,  /* sizes beyond what the kernels hold on chip (e.g. M0 > 128) */
+    AVQ_ECUDA = -3,         /* a CUDA launch or runtime call failed */
+    AVQ_ETIMEOUT = -4,      /* a bounded device-side wait ran out (reported by avq_device_status) */
+    AVQ_EWORKSPACE = -5     /* workspace missing or smaller than the *_workspace_bytes() answer */
+} avq_status;
+
+/*
+ * Workspace needed by avq_precompute for `s` (bytes, a multiple of 256;
+ * 0 for invalid shapes). The workspace holds the device status word read by
+ * avq_device_status and per-head scratch of the aggregation.
+ */
+size_t avq_precompute_workspace_bytes(const avq_shape* s);
+
+/*
+ * Fused full-tree VQ precompute (paper §4.2; papernotes, Key Designs 2;
+ * paper Table 1, rows "VQ assignment" and "Value aggregation").
+ *
+ * For every key k of head (b,h):
+ *   p*(k)  = argmin_p ||K_k - C_p||^2 over the M0 parents (squared Euclidean
+ *            distance; ties to the lowest index), distance kept;
+ *   leaf   = the child M0 + p*C + c of p* with the smallest distance if that
+ *            distance is STRICTLY smaller than the kept parent distance
+ *            (lowest c among equal children), else p*;
+ *   assign[b,h,k] = leaf.
+ * Decisions are those of exact fp64 arithmetic on the stored values: the
+ * kernels filter with fp32 distances and a rigorous error bound and re-decide
+ * in fp64 whenever the bound does not separate the candidates.
+ *   counts[b,h,p] / vsum[b,h,p,:] : number / sum of V rows of ALL keys with
+ *                                   p*(k) = p (the parent's whole cluster);
+ *   counts[b,h,j] / vsum[b,h,j,:] : for a child j, only the keys whose leaf is j.
+ * vsum is accumulated in fp32 (summation order unspecified).
+ *
+ * K, V, codebook: device, read only. assign, counts, vsum: device, written
+ * (zeroed by the call). workspace: device, >= avq_precompute_workspace_bytes(s).
+ */
+int avq_precompute(const avq_shape* s, const void* K, const void* V, const void* codebook,
+                   int32_t* assign, int32_t* counts, float* vsum,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace needed by avq_attention for `s`, P and tile (bytes, multiple of
+ * 256; 0 for invalid arguments). It holds the device status word and
+ * per-head tables derived from counts/vsum each call.
+ */
+size_t avq_attention_workspace_bytes(const avq_shape* s, int P, int tile);
+
+/*
+ * Tiled adaptive attention (paper §4.3; papernotes, Key Designs 3).
+ *
+ * Queries of head (b,h) are cut into consecutive tiles of `tile` rows
+ * (tile in {64, 128}; a partial last tile is masked). For each query i:
+ *   S_ij = scale * Q_i . C_j  (the paper writes exp(Q C^T), scale folded in Q);
+ *   parent attention  A_ip = exp(S_ip - m_i), Zbar_i = sum_p A_ip n_p, over
+ *   parents with n_p > 0 (m_i their largest logit).
+ * For each tile I:
+ *   importance w_p(I) = sum_{i in I} A_ip n_p / Zbar_i ("Codeword importance");
+ *   selected[b,h,t,:] = the P parents of largest w, by descending w, ties to
+ *   the lower index ("Child spawning"); 0 <= P <= M0.
+ * Output, with one shift for all terms of query i:
+ *   Xbar_i = sum_p e^{S_ip} vsum_p
+ *          + sum_{p selected} sum_c (e^{S_ic} - e^{S_ip}) vsum_{p,c}
+ *   Zbar_i likewise with counts (the DeltaA correction of papernotes, Key
+ *   Designs 3);  O_i = Xbar_i / Zbar_i, stored in Q's dtype.
+ * counts/vsum are avq_precompute's outputs for the same codebook.
+ *
+ * Q, codebook, counts, vsum: device, read only. O, selected: device,
+ * written. selected may be NULL when P == 0. workspace: device,
+ * >= avq_attention_workspace_bytes(s, P, tile).
+ */
+int avq_attention(const avq_shape* s, const void* Q, const void* codebook,
+                  const int32_t* counts, const float* vsum, int P, int tile, float scale,
+                  void* O, int32_t* selected, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/*
+ * Blocking: waits for `stream`, then reads the status word that kernels of
+ * earlier calls using `workspace` left there (AVQ_OK, or AVQ_ETIMEOUT when a
+ * bounded device-side wait ran out) and clears it. Returns AVQ_ECUDA if the
+ * stream reports an error.
+ */
+int avq_device_status(void* workspace, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* avq_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int avq_version(void);
+
+/*
+ * Number of CUDA kernels this library has enqueued in this process so far
+ * (all calls, all devices; host-side counter, thread-safe). Lets a caller
+ * count the library's launches inside a timed region.
+ */
+uint64_t avq_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AVQ_B200_H */

@@ -1,0 +1,121 @@
+"""Parity harness: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Acceptance (per the method's statement of tolerances, and readings R14 of
+the design notes):
+* ``assign`` and ``counts`` bit-exact;
+* ``vsum`` within 1e-5 of the per-codeword sum of |V| (fp32 accumulation);
+* ``selected``: every parent whose normalised oracle score lies more than
+  1e-6 above the P-th score is selected, none lying more than 1e-6 below it
+  is, and consecutive entries never invert the oracle's order by more than
+  1e-6; a tile whose GPU set differs from the oracle's (only possible inside
+  the band) is counted as a tie-band tile and its outputs are compared with
+  the oracle re-run on the GPU's selection;
+* ``O`` max-abs error <= 2e-3 (fp32 inputs) or 2e-2 (bf16 inputs).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from adaptive_vector_quantized_avq_b200 import binding as bd
+from adaptive_vector_quantized_avq_b200 import synthetic as syn
+
+BAND = 1e-6
+O_TOL = {"f32": 2e-3, "bf16": 2e-2}
+VSUM_REL = 1e-5
+
+
+def to_device(arr: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
+    if dtype == "bf16":
+        return torch.from_numpy(arr.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+
+
+def from_device(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return syn.bf16_bits_to_f64(t.view(torch.int16).cpu().numpy().view(np.uint16))
+    return t.cpu().numpy()
+
+
+def run_gpu(wl: syn.Workload, inp: syn.Inputs, Ps, device="cuda"):
+    dt = wl.dtype
+    K, V, Q, cb = (to_device(getattr(inp, n), dt, device) for n in ("K", "V", "Q", "codebook"))
+    assign, counts, vsum = bd.precompute(K, V, cb, wl.M0, wl.C)
+    att = {}
+    for P in Ps:
+        O, sel = bd.attention(Q, cb, counts, vsum, wl.M0, wl.C, P, wl.tile, wl.softmax_scale)
+        att[P] = (O, sel)
+    torch.cuda.synchronize()
+    return {"assign": assign.cpu().numpy(), "counts": counts.cpu().numpy(),
+            "vsum": vsum.cpu().numpy(),
+            "att": {P: (from_device(O), sel.cpu().numpy()) for P, (O, sel) in att.items()}}
+
+
+class Report(dict):
+    pass
+
+
+def check_precompute(wl, inp, gpu, ora, oracle) -> Report:
+    rep = Report()
+    bad = np.nonzero(gpu["assign"] != ora["assign"])
+    assert bad[0].size == 0, f"{wl.name}: {bad[0].size} assignments differ, first at {[b[0] for b in bad]}: " \
+                             f"gpu {gpu['assign'][tuple(b[0] for b in bad)]} oracle {ora['assign'][tuple(b[0] for b in bad)]}"
+    assert np.array_equal(gpu["counts"], ora["counts"]), f"{wl.name}: counts differ"
+    # per-codeword sum of |V| from the oracle itself (same assignment rule)
+    absV = np.abs(inp.f64("V"))
+    abs_sum = oracle.precompute(inp.f64("K"), absV, inp.f64("codebook"), wl.M0, wl.C)["vsum"]
+    err = np.abs(gpu["vsum"] - ora["vsum"])
+    lim = VSUM_REL * abs_sum + 1e-30
+    worst = float((err / np.maximum(abs_sum, 1e-30)).max()) if err.size else 0.0
+    assert np.all(err <= lim), f"{wl.name}: vsum error {worst:.3g} of sum|V| exceeds {VSUM_REL}"
+    rep["vsum_rel_err"] = worst
+    return rep
+
+
+def check_selection(sel_gpu, sel_ora, score, P):
+    """Returns True when the GPU set equals the oracle's; raises outside the band."""
+    if P == 0:
+        return True
+    kth = np.sort(score)[::-1][P - 1]
+    g = set(int(x) for x in sel_gpu)
+    assert len(g) == P and all(0 <= x < score.size for x in g), f"invalid selection {sel_gpu}"
+    sure_in = set(np.nonzero(score > kth + BAND)[0].tolist())
+    sure_out = set(np.nonzero(score < kth - BAND)[0].tolist())
+    assert sure_in <= g, f"selection misses {sorted(sure_in - g)} (scores {score[list(sure_in - g)]}, kth {kth})"
+    assert not (g & sure_out), f"selection takes {sorted(g & sure_out)} below the band"
+    for a, b in zip(sel_gpu[:-1], sel_gpu[1:]):
+        assert score[a] >= score[b] - BAND, f"order inverted: {a} ({score[a]}) before {b} ({score[b]})"
+    return g == set(int(x) for x in sel_ora)
+
+
+def check_attention(wl, inp, P, gpu_O, gpu_sel, counts, vsum, oracle, tile_ids=None) -> Report:
+    """Compare all tiles (tile_ids None) or the listed global tile ids."""
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    T = wl.tile
+    ntiles = wl.ntiles
+    Q = inp.f64("Q")
+    cb = inp.f64("codebook")
+    ids = np.arange(B * H * ntiles) if tile_ids is None else np.asarray(tile_ids)
+    ora = oracle.attention(Q, cb, counts, vsum, wl.M0, wl.C, P, T, wl.softmax_scale, tile_ids=ids)
+    gsel = gpu_sel.reshape(B * H * ntiles, P)[ids] if P > 0 else np.zeros((ids.size, 0), np.int32)
+    band_tiles = []
+    for j in range(ids.size):
+        if not check_selection(gsel[j], ora["selected"][j], ora["score"][j], P):
+            band_tiles.append(j)
+    O_ref = ora["O"].copy()
+    if band_tiles:
+        forced = oracle.attention(Q, cb, counts, vsum, wl.M0, wl.C, P, T, wl.softmax_scale,
+                                  tile_ids=ids[band_tiles], forced=gsel[band_tiles])
+        O_ref[band_tiles] = forced["O"]
+    # gather the GPU rows of the listed tiles
+    Og = gpu_O.reshape(B * H, N, d)
+    err = 0.0
+    for j, g in enumerate(ids):
+        bh, t = divmod(int(g), ntiles)
+        r0, r1 = t * T, min(N, (t + 1) * T)
+        e = np.abs(Og[bh, r0:r1] - O_ref[j, : r1 - r0]).max() if r1 > r0 else 0.0
+        err = max(err, float(e))
+    tol = O_TOL[wl.dtype]
+    assert err <= tol, f"{wl.name} P={P}: O max-abs error {err:.3g} > {tol}"
+    assert np.isfinite(Og).all(), "non-finite output"
+    return Report(O_maxabs=err, tiles=int(ids.size), tie_band_tiles=len(band_tiles))
