@@ -21,7 +21,7 @@ from . import build as _build
 AVQ_F32, AVQ_BF16 = 0, 1
 AVQ_OK = 0
 _STATUS = {0: "AVQ_OK", -1: "AVQ_EINVAL", -2: "AVQ_EUNSUPPORTED", -3: "AVQ_ECUDA",
-           -4: "AVQ_ETIMEOUT", -5: "AVQ_EWORKSPACE"}
+           -4: "AVQ_ETIMEOUT", -5: "AVQ_EWORKSPACE", -6: "AVQ_ERANGE"}
 
 # every symbol include/avq.h declares (checked by the tests)
 EXPORTS = ("avq_precompute_workspace_bytes", "avq_precompute", "avq_attention_workspace_bytes",

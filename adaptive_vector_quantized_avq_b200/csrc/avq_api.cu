@@ -20,6 +20,11 @@ cudaError_t launch_attention_simt(const avq_shape& s, const void* Q, const void*
                                   const int32_t* counts, const float* vsum, int P, int tile,
                                   float scale, void* O, int32_t* selected, cudaStream_t st);
 size_t attention_simt_smem(const avq_shape& s);
+bool attention_tc_supported(const avq_shape& s, int tile);
+size_t attention_tc_workspace(const avq_shape& s);
+cudaError_t launch_attention_tc(const avq_shape& s, const void* Q, const void* cb, const int32_t* counts,
+                                const float* vsum, int P, float scale, void* O, int32_t* selected,
+                                void* vtab, StatusBlock* status, cudaStream_t st);
 }  // namespace avq
 
 using namespace avq;
@@ -65,6 +70,7 @@ const char* avq_status_string(int st) {
         case AVQ_ECUDA: return "AVQ_ECUDA: a CUDA call failed";
         case AVQ_ETIMEOUT: return "AVQ_ETIMEOUT: a bounded device-side wait ran out";
         case AVQ_EWORKSPACE: return "AVQ_EWORKSPACE: workspace missing or too small";
+        case AVQ_ERANGE: return "AVQ_ERANGE: a child logit exceeded its query's parent maximum by more than 60";
         default: return "unknown avq status";
     }
 }
@@ -99,7 +105,9 @@ int avq_precompute(const avq_shape* s, const void* K, const void* V, const void*
 size_t avq_attention_workspace_bytes(const avq_shape* s, int P, int tile) {
     if (check_shape(s) != AVQ_OK) return 0;
     if (P < 0 || P > s->M0 || (tile != 64 && tile != 128)) return 0;
-    return kStatusBytes;
+    size_t n = kStatusBytes;
+    if (attention_tc_supported(*s, tile)) n += attention_tc_workspace(*s);
+    return n;
 }
 
 int avq_attention(const avq_shape* s, const void* Q, const void* codebook, const int32_t* counts,
@@ -118,8 +126,14 @@ int avq_attention(const avq_shape* s, const void* Q, const void* codebook, const
     if (rc != AVQ_OK) return rc;
     if (s->N == 0) return AVQ_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_attention_simt(*s, Q, codebook, counts, vsum, P, tile, scale, O,
-                                          selected, st);
+    cudaError_t e;
+    if (attention_tc_supported(*s, tile)) {
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        e = launch_attention_tc(*s, Q, codebook, counts, vsum, P, scale, O, selected, ws + kStatusBytes,
+                                reinterpret_cast<StatusBlock*>(ws), st);
+    } else {
+        e = launch_attention_simt(*s, Q, codebook, counts, vsum, P, tile, scale, O, selected, st);
+    }
     return e == cudaSuccess ? AVQ_OK : AVQ_ECUDA;
 }
 

@@ -67,7 +67,10 @@ typedef enum {
     AVQ_EUNSUPPORTED = -2,  /* sizes beyond what the kernels hold on chip (e.g. M0 > 128) */
     AVQ_ECUDA = -3,         /* a CUDA launch or runtime call failed */
     AVQ_ETIMEOUT = -4,      /* a bounded device-side wait ran out (reported by avq_device_status) */
-    AVQ_EWORKSPACE = -5     /* workspace missing or smaller than the *_workspace_bytes() answer */
+    AVQ_EWORKSPACE = -5,    /* workspace missing or smaller than the *_workspace_bytes() answer */
+    AVQ_ERANGE = -6         /* (device status) a child logit exceeded the largest non-empty parent
+                               logit of its query by more than 60 (natural-log units): the
+                               common-shift weights may overflow fp32 for that query */
 } avq_status;
 
 /*
@@ -140,9 +143,10 @@ int avq_attention(const avq_shape* s, const void* Q, const void* codebook,
 
 /*
  * Blocking: waits for `stream`, then reads the status word that kernels of
- * earlier calls using `workspace` left there (AVQ_OK, or AVQ_ETIMEOUT when a
- * bounded device-side wait ran out) and clears it. Returns AVQ_ECUDA if the
- * stream reports an error.
+ * earlier calls using `workspace` left there (AVQ_OK; AVQ_ETIMEOUT when a
+ * bounded device-side wait ran out; AVQ_ERANGE, see above) and clears it.
+ * Returns AVQ_ECUDA if the stream reports an error. A workspace must be
+ * zero-filled before its first use.
  */
 int avq_device_status(void* workspace, void* stream);
 

@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_version_and_status_strings(L):
     assert bd.avq_version() >= 100
-    for code in (0, -1, -2, -3, -4, -5):
+    for code in (0, -1, -2, -3, -4, -5, -6):
         assert bd.avq_status_string(code).startswith(bd._STATUS[code])
 
 
