@@ -21,6 +21,10 @@ cudaError_t launch_attention_simt(const avq_shape& s, const void* Q, const void*
                                   float scale, void* O, int32_t* selected, cudaStream_t st);
 size_t attention_simt_smem(const avq_shape& s);
 bool attention_tc_supported(const avq_shape& s, int tile);
+bool precompute_tc_supported(const avq_shape& s);
+cudaError_t launch_precompute_tc(const avq_shape& s, const void* K, const void* V, const void* cb,
+                                 int32_t* assign, int32_t* counts, float* vsum, StatusBlock* status,
+                                 cudaStream_t st);
 size_t attention_tc_workspace(const avq_shape& s);
 cudaError_t launch_attention_tc(const avq_shape& s, const void* Q, const void* cb, const int32_t* counts,
                                 const float* vsum, int P, float scale, void* O, int32_t* selected,
@@ -98,7 +102,12 @@ int avq_precompute(const avq_shape* s, const void* K, const void* V, const void*
     if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * BH * Mtot, st) != cudaSuccess) return AVQ_ECUDA;
     if (cudaMemsetAsync(vsum, 0, sizeof(float) * BH * Mtot * s->d, st) != cudaSuccess) return AVQ_ECUDA;
     if (s->N == 0) return AVQ_OK;
-    cudaError_t e = launch_precompute_simt(*s, K, V, codebook, assign, counts, vsum, st);
+    cudaError_t e;
+    if (precompute_tc_supported(*s))
+        e = launch_precompute_tc(*s, K, V, codebook, assign, counts, vsum,
+                                 static_cast<StatusBlock*>(workspace), st);
+    else
+        e = launch_precompute_simt(*s, K, V, codebook, assign, counts, vsum, st);
     return e == cudaSuccess ? AVQ_OK : AVQ_ECUDA;
 }
 

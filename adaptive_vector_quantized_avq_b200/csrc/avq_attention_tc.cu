@@ -460,36 +460,6 @@ __global__ void vsum_to_bf16_kernel(const float4* __restrict__ src, uint2* __res
     }
 }
 
-// ------------------------------------------------------------ tensor maps
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
-// 3-D bf16 tensor [n2][n1][n0] (n0 innermost), box {64, box1, 1}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box1) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {n0, n1, n2};
-    const cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
-    const cuuint32_t box[3] = {64, box1, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int C>
 cudaError_t launch_tc(const avq_shape& s, const void* Q, const void* cb, const int32_t* counts, int P,
                       float scale, void* O, int32_t* selected, const void* vtab, StatusBlock* status,
@@ -498,8 +468,8 @@ cudaError_t launch_tc(const avq_shape& s, const void* Q, const void* cb, const i
     const int Mtot = s.M0 * (1 + s.C);
     const int M0p = (s.M0 + 15) & ~15;
     CUtensorMap tq, to, tcb, tvt;
-    if (!make_map(&tq, Q, D, s.N, BH, kTile) || !make_map(&to, O, D, s.N, BH, kTile) ||
-        !make_map(&tcb, cb, D, Mtot, s.H, M0p) || !make_map(&tvt, vtab, D, Mtot, BH, M0p))
+    if (!make_tma_bf16_3d(&tq, Q, D, s.N, BH, kTile) || !make_tma_bf16_3d(&to, O, D, s.N, BH, kTile) ||
+        !make_tma_bf16_3d(&tcb, cb, D, Mtot, s.H, M0p) || !make_tma_bf16_3d(&tvt, vtab, D, Mtot, BH, M0p))
         return cudaErrorInvalidValue;
     TcAttnParams prm;
     prm.BH = BH;

@@ -19,6 +19,11 @@
 #include <stdint.h>
 
 namespace avq {
+
+// 3-D bf16 tensor [n2][n1][n0] (n0 innermost, n0*2 bytes a multiple of 16),
+// box {64, box1, 1}, 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_tma_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t box1);
+
 namespace sm100 {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

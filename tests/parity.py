@@ -38,16 +38,27 @@ def from_device(t: torch.Tensor) -> np.ndarray:
 
 
 def run_gpu(wl: syn.Workload, inp: syn.Inputs, Ps, device="cuda"):
+    """Both calls through the C ABI; also checks the device status words
+    (no timeout, no range flag) and returns the fp64 re-decision counters."""
     dt = wl.dtype
     K, V, Q, cb = (to_device(getattr(inp, n), dt, device) for n in ("K", "V", "Q", "codebook"))
-    assign, counts, vsum = bd.precompute(K, V, cb, wl.M0, wl.C)
+    shape = bd.make_shape(wl.B, wl.H, wl.N, wl.d, wl.M0, wl.C, K.dtype)
+    ws_pre = bd.workspace(bd.avq_precompute_workspace_bytes(shape), K.device)
+    assign, counts, vsum = bd.precompute(K, V, cb, wl.M0, wl.C, ws=ws_pre)
+    torch.cuda.synchronize()
+    diag = ws_pre[:16].view(torch.int32).cpu().numpy()
+    st = bd.avq_device_status(ws_pre)
+    assert st == 0, f"precompute device status {st}"
     att = {}
     for P in Ps:
-        O, sel = bd.attention(Q, cb, counts, vsum, wl.M0, wl.C, P, wl.tile, wl.softmax_scale)
+        ws_att = bd.workspace(bd.avq_attention_workspace_bytes(shape, P, wl.tile), K.device)
+        O, sel = bd.attention(Q, cb, counts, vsum, wl.M0, wl.C, P, wl.tile, wl.softmax_scale, ws=ws_att)
+        st = bd.avq_device_status(ws_att)
+        assert st == 0, f"attention device status {st} (P={P})"
         att[P] = (O, sel)
     torch.cuda.synchronize()
     return {"assign": assign.cpu().numpy(), "counts": counts.cpu().numpy(),
-            "vsum": vsum.cpu().numpy(),
+            "vsum": vsum.cpu().numpy(), "redecided": (int(diag[2]), int(diag[3])),
             "att": {P: (from_device(O), sel.cpu().numpy()) for P, (O, sel) in att.items()}}
 
 
@@ -69,6 +80,7 @@ def check_precompute(wl, inp, gpu, ora, oracle) -> Report:
     worst = float((err / np.maximum(abs_sum, 1e-30)).max()) if err.size else 0.0
     assert np.all(err <= lim), f"{wl.name}: vsum error {worst:.3g} of sum|V| exceeds {VSUM_REL}"
     rep["vsum_rel_err"] = worst
+    rep["fp64_redecided_parent_child"] = gpu.get("redecided")
     return rep
 
 
