@@ -14,7 +14,7 @@ _BINDING_NAMES = {
     "precompute", "attention", "workspace", "AVQError", "make_shape", "lib", "library_path",
     "avq_precompute", "avq_attention", "avq_precompute_workspace_bytes",
     "avq_attention_workspace_bytes", "avq_device_status", "avq_status_string", "avq_version",
-    "avq_kernel_launches",
+    "avq_kernel_launches", "avq_attention_noalloc",
     "EXPORTS",
 }
 

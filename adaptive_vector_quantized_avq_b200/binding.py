@@ -26,7 +26,7 @@ _STATUS = {0: "AVQ_OK", -1: "AVQ_EINVAL", -2: "AVQ_EUNSUPPORTED", -3: "AVQ_ECUDA
 # every symbol include/avq.h declares (checked by the tests)
 EXPORTS = ("avq_precompute_workspace_bytes", "avq_precompute", "avq_attention_workspace_bytes",
            "avq_attention", "avq_device_status", "avq_status_string", "avq_version",
-           "avq_kernel_launches")
+           "avq_kernel_launches", "avq_attention_noalloc")
 
 
 class AVQError(RuntimeError):
@@ -74,6 +74,9 @@ def lib() -> ctypes.CDLL:
         L.avq_status_string.restype = ctypes.c_char_p
         L.avq_version.argtypes = []
         L.avq_version.restype = i32
+        L.avq_attention_noalloc.argtypes = [shp, vp, vp, vp, vp, i32, i32, ctypes.c_float, vp, vp,
+                                            vp, vp]
+        L.avq_attention_noalloc.restype = i32
         L.avq_kernel_launches.argtypes = []
         L.avq_kernel_launches.restype = ctypes.c_uint64
         _LIB = L
@@ -136,6 +139,13 @@ def avq_attention(shape, Q, codebook, counts, vsum, P, tile, scale, O, selected,
     return lib().avq_attention(ctypes.byref(shape), _ptr(Q), _ptr(codebook), _ptr(counts),
                                _ptr(vsum), P, tile, float(scale), _ptr(O), _ptr(selected),
                                _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def avq_attention_noalloc(shape, Q, codebook, counts, vsum, P, tile, scale, O, selected,
+                          device_status=None, stream=None) -> int:
+    return lib().avq_attention_noalloc(ctypes.byref(shape), _ptr(Q), _ptr(codebook), _ptr(counts),
+                                       _ptr(vsum), P, tile, float(scale), _ptr(O), _ptr(selected),
+                                       _ptr(device_status), _stream(stream))
 
 
 def avq_device_status(workspace, stream=None) -> int:

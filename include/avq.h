@@ -142,6 +142,33 @@ int avq_attention(const avq_shape* s, const void* Q, const void* codebook,
                   void* stream);
 
 /*
+ * avq_attention for callers that cannot allocate device memory (a host
+ * framework that owns all device allocations and forbids its plugins to call
+ * cudaMalloc, or latency-bound code that cannot afford cudaMalloc's implicit
+ * device synchronisation). The paper has no counterpart: this is a property
+ * of the library's interface only. Same arguments, results and errors as
+ * avq_attention, with no workspace: the scratch lives in a fixed 8 MiB array
+ * of device memory owned by the library (on every GPU that loads it, until
+ * the process exits).
+ *
+ * - Problems whose scratch, 256 + B*H*M0*(1+C)*d*2 bytes, exceeds 8 MiB are
+ *   rejected with AVQ_EWORKSPACE before anything is enqueued.
+ * - The first call on a device looks the array's device address up (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture on the device.
+ * - All calls on a device share the array and it keeps the last call's
+ *   contents; calls whose work overlaps on the GPU (different streams or host
+ *   threads) race on it and must be serialised by the caller.
+ * - device_status (device pointer to one int32, may be NULL) receives this
+ *   call's device status word (AVQ_OK, AVQ_ETIMEOUT or AVQ_ERANGE), written
+ *   on `stream`.
+ * - Allocates nothing: no cudaMalloc/cudaFree and no allocating library call.
+ */
+int avq_attention_noalloc(const avq_shape* s, const void* Q, const void* codebook,
+                          const int32_t* counts, const float* vsum, int P, int tile, float scale,
+                          void* O, int32_t* selected, int32_t* device_status, void* stream);
+
+/*
  * Blocking: waits for `stream`, then reads the status word that kernels of
  * earlier calls using `workspace` left there (AVQ_OK; AVQ_ETIMEOUT when a
  * bounded device-side wait ran out; AVQ_ERANGE, see above) and clears it.
