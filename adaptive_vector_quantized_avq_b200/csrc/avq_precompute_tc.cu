@@ -2,8 +2,13 @@
 // bf16 inputs (paper §4.2; papernotes, Key Designs 2; paper Table 1 rows
 // "VQ assignment" and "Value aggregation").
 //
-// Persistent: one 128-thread CTA per SM walks a contiguous range of 128-key
-// tiles (head-major). Thread r owns key r of the tile and TMEM lane r.
+// Persistent: one 256-thread CTA per SM walks a contiguous range of 128-key
+// tiles (head-major). Key r of a tile is handled by the thread pair r and
+// r + 128 (halves h = 0, 1): each half holds half of the key's dimensions and
+// scans half of the parents. The pair combines its parent scans through shared
+// memory (both threads then hold the same nearest parent); for the children,
+// half 1 publishes its partial distances and half 0 completes them, decides
+// and writes the outputs. TMEM lane r holds key r's dot products.
 //
 // Per head (when the range enters it): TMA brings the parent codewords (the
 // B operand), cp.async brings the C*M0 child codewords into a shared-memory
@@ -16,14 +21,15 @@
 //   1. TMA brings K and V (two stages, issued two tiles ahead).
 //   2. MMA  S = K C_par^T  (M=128, N=M0p, K=d) into one of two TMEM buffers,
 //      issued one tile ahead.
-//   3. a1: D~_p = ||k||^2 + ||C_p||^2 - 2 S_p in fp32; the smallest and the
-//      runner-up. If they are not separated by the error bound of this
-//      expanded form, the parents within the band are re-decided with the
-//      exact fp64 distance summed in index order.
+//   3. a1: v_p = ||C_p||^2 - 2 S_p (the expanded distance minus ||k||^2) in
+//      fp32; the smallest and the runner-up. If they are not separated by the
+//      error bound of this expanded form, the parents within the band are
+//      re-decided with the exact fp64 distance summed in index order.
 //   4. a2: the kept parent and its C children by the direct form
-//      sum_j (k_j - c_j)^2 in fp32 (relative error <= (d+4)u); a candidate
-//      wins only when strictly closer (parent first, lowest child index among
-//      equals); the band the bound cannot separate is re-decided in fp64.
+//      sum_j (k_j - c_j)^2 in fp32 (packed f32x2 arithmetic, relative error
+//      <= (d+4)u); a candidate wins only when strictly closer (parent first,
+//      lowest child index among equals); the band the bound cannot separate
+//      is re-decided in fp64.
 //   5. a3: assign written; counts in shared memory; the key's V row is added
 //      to the parent's and (when the key moved) the child's value sum with
 //      warp-wide coalesced fp32 vector reductions (one 256-byte row per
@@ -39,10 +45,12 @@ using namespace sm100;
 namespace {
 
 constexpr int kTile = 128;
+constexpr int kThreads = 256;
 constexpr uint32_t kRegion = 128 * 128;
 
 struct TcPreParams {
     int BH, H, N, M0, M0p, Mtot, ntiles, total_tiles;
+    const uint16_t* K;          // [BH, N, D] bf16 (exact re-decisions read keys here)
     const uint16_t* codebook;   // [H, Mtot, D] bf16
     int32_t* assign;            // [BH, N]
     int32_t* counts;            // [BH, Mtot]
@@ -69,35 +77,61 @@ __device__ __forceinline__ uint32_t ch_off(int i, int p, int j) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Squared distance of the key (fp32 registers) to a bf16 row in shared memory
-// whose chunk j lives at byte offset chunk_off(j); two interleaved fp32
-// accumulators, each term (k - c)^2 rounded once by the fused multiply-add.
-template <int D, typename F>
-__device__ __forceinline__ float direct_dist(const float (&k)[D], const uint8_t* row_base, F chunk_off) {
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-        const uint4 w = *reinterpret_cast<const uint4*>(row_base + chunk_off(j));
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float t0 = __fsub_rn(k[8 * j + 2 * e], bf_lo(ww[e]));
-            const float t1 = __fsub_rn(k[8 * j + 2 * e + 1], bf_hi(ww[e]));
-            a0 = __fmaf_rn(t0, t0, a0);
-            a1 = __fmaf_rn(t1, t1, a1);
-        }
-    }
-    return __fadd_rn(a0, a1);
+// packed fp32 pairs (sm_100 f32x2 arithmetic, round-to-nearest per lane)
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t pk2(float lo, float hi) {
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ f2_t bf2_to_f2(uint32_t w) { return pk2(bf_lo(w), bf_hi(w)); }
+__device__ __forceinline__ f2_t sub2(f2_t a, f2_t b) {
+    f2_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
+    f2_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ float hsum2(f2_t a) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a));
+    return __fadd_rn(lo, hi);
 }
 
-// Exact fp64 distance of the key (fp32 registers hold exact bf16 values) to a
-// global bf16 codeword, terms in index order, no fused operations.
+// Partial squared distance over this half's NC 16-byte chunks (chunk index
+// offset j0) of the key (packed pairs) to a bf16 row in shared memory whose
+// chunk j lives at chunk_off(j); each term (k - c)^2 rounded once (fused).
+template <int NC, typename F>
+__device__ __forceinline__ float half_dist(const f2_t (&k2)[NC * 4], const uint8_t* row_base, int j0,
+                                           F chunk_off) {
+    f2_t a = 0ull, b = 0ull;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(row_base + chunk_off(j0 + j));
+        const f2_t t0 = sub2(k2[4 * j + 0], bf2_to_f2(w.x));
+        const f2_t t1 = sub2(k2[4 * j + 1], bf2_to_f2(w.y));
+        const f2_t t2 = sub2(k2[4 * j + 2], bf2_to_f2(w.z));
+        const f2_t t3 = sub2(k2[4 * j + 3], bf2_to_f2(w.w));
+        a = fma2(t0, t0, a);
+        b = fma2(t1, t1, b);
+        a = fma2(t2, t2, a);
+        b = fma2(t3, t3, b);
+    }
+    return __fadd_rn(hsum2(a), hsum2(b));
+}
+
+// Exact fp64 distance between two global bf16 rows, terms in index order,
+// no fused operations.
 template <int D>
-__device__ __noinline__ double exact_dist_reg(const float* k, const uint16_t* c) {
+__device__ __noinline__ double exact_dist_glob(const uint16_t* k, const uint16_t* c) {
     double s = 0.0;
     for (int j = 0; j < D; ++j) {
+        const double kj = (double)__uint_as_float((uint32_t)__ldg(k + j) << 16);
         const double cj = (double)__uint_as_float((uint32_t)__ldg(c + j) << 16);
-        const double t = __dsub_rn((double)k[j], cj);
+        const double t = __dsub_rn(kj, cj);
         s = __dadd_rn(s, __dmul_rn(t, t));
     }
     return s;
@@ -112,12 +146,13 @@ __device__ __forceinline__ void red_v4(float* addr, float a, float b, float c, f
 }
 
 template <int D, int C>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmCB, const TcPreParams p) {
     constexpr int KH = D / 64;
     constexpr uint32_t IMG = KH * kRegion;
     constexpr int KSTEPS = D / 16;
+    constexpr int NCH = D / 16;          // 16-byte chunks per half row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = align1024p(smem_raw);
     uint8_t* sK0 = base;                     // K stages: sK0 + s*IMG
@@ -126,15 +161,22 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     uint8_t* sCh = base + 5 * IMG;           // children image [M0*C rows x D] bf16
     const size_t ch_bytes = (size_t)p.M0 * C * D * 2;
     float* sCn = reinterpret_cast<float*>(sCh + ((ch_bytes + 15) & ~size_t(15)));   // [128]
-    int* sCnt = reinterpret_cast<int*>(sCn + 128);                                     // [Mtot]
-    int* sPar = sCnt + ((p.Mtot + 3) & ~3);                                            // [128]
-    int* sLeaf = sPar + 128;                                                           // [128]
-    float* sRed = reinterpret_cast<float*>(sLeaf + 128);                               // [4]
-    uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(sRed + 4) + 7) & ~uintptr_t(7));
+    float* sKn = sCn + 128;                  // [2][128] partial ||k||^2
+    float* sBest = sKn + 256;                // [2][128]
+    float* sSecond = sBest + 256;            // [2][128]
+    int* sIdx = reinterpret_cast<int*>(sSecond + 256);       // [2][128]
+    float* sDist = reinterpret_cast<float*>(sIdx + 256);     // [C+1][128] partial distances of half 1
+    int* sPar = reinterpret_cast<int*>(sDist + (C + 1) * 128);       // [128]
+    int* sLeaf = sPar + 128;                 // [128]
+    float* sRed = reinterpret_cast<float*>(sLeaf + 128);     // [8]
+    int* sCnt = reinterpret_cast<int*>(sRed + 8);            // [Mtot]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(
+        (reinterpret_cast<uintptr_t>(sCnt + p.Mtot) + 7) & ~uintptr_t(7));
     // bars: 0,1 = K stage; 2,3 = V stage; 4,5 = MMA buffer; 6 = head
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 7);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = tid & 127, half = tid >> 7;
     const int g0 = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
     const int g1 = (int)(((long long)(blockIdx.x + 1) * p.total_tiles) / gridDim.x);
 
@@ -149,15 +191,16 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmCB);
     }
-    for (int i = tid; i < p.Mtot; i += 128) sCnt[i] = 0;
+    for (int i = tid; i < p.Mtot; i += kThreads) sCnt[i] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *sTmem;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t idesc = idesc_bf16_f32(128, p.M0p, false);
     const float eps_dir = dist_eps(D);
-    // expanded-form bound factor (see DESIGN notes): 2 * (5d + 8) * 2^-24
+    // expanded-form bound factor: 2 * (5d + 8) * 2^-24 (per distance, times
+    // ||k||^2 + max ||C_p||^2)
     const float c_exp = 2.f * (5.f * D + 8.f) * 5.9604644775390625e-08f;
 
     uint32_t kph = 0, vph = 0, mph = 0, hph = 0;   // phase bit of stage s = bit s
@@ -188,7 +231,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         return true;
     };
     auto flush_counts = [&](int bh) {
-        for (int i = tid; i < p.Mtot; i += 128) {
+        for (int i = tid; i < p.Mtot; i += kThreads) {
             const int c = sCnt[i];
             if (c) {
                 atomicAdd(p.counts + (size_t)bh * p.Mtot + i, c);
@@ -207,7 +250,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         const int s = it & 1;
         const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
         const int rows = min(kTile, p.N - t * kTile);
-        const bool valid = tid < rows;
+        const bool valid = r < rows;
 
         if (bh != cur_bh) {
             // flush the previous head's counts, load the new head's codewords
@@ -219,7 +262,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                     for (int kh = 0; kh < KH; ++kh) tma_load_3d(sB1 + kh * kRegion, &tmCB, &bars[6], kh * 64, 0, h);
                 }
                 const uint16_t* chg = p.codebook + ((size_t)h * p.Mtot + p.M0) * D;
-                for (int idx = tid; idx < p.M0 * C * (D / 8); idx += 128) {
+                for (int idx = tid; idx < p.M0 * C * (D / 8); idx += kThreads) {
                     const int i = idx / (D / 8), j = idx % (D / 8);
                     cp_async_16(sCh + ch_off<D>(i, i / C, j), chg + (size_t)i * D + j * 8);
                 }
@@ -233,7 +276,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                         cn = __fmaf_rn(c, c, cn);
                     }
                 }
-                sCn[tid] = cn;
+                if (tid < 128) sCn[tid] = cn;
                 float mx = cn;
 #pragma unroll
                 for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -259,22 +302,23 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
 
-        // key row -> fp32 registers; ||k||^2
-        float k[D];
+        // this half of the key row -> packed fp32 pairs; partial ||k||^2
+        f2_t k2[NCH * 4];
         {
             const uint8_t* kimg = sK0 + s * IMG;
+            f2_t acc = 0ull;
 #pragma unroll
-            for (int j = 0; j < D / 8; ++j) {
-                const uint4 w = *reinterpret_cast<const uint4*>(kimg + swz_off(tid, j));
-                k[8 * j + 0] = bf_lo(w.x); k[8 * j + 1] = bf_hi(w.x);
-                k[8 * j + 2] = bf_lo(w.y); k[8 * j + 3] = bf_hi(w.y);
-                k[8 * j + 4] = bf_lo(w.z); k[8 * j + 5] = bf_hi(w.z);
-                k[8 * j + 6] = bf_lo(w.w); k[8 * j + 7] = bf_hi(w.w);
+            for (int j = 0; j < NCH; ++j) {
+                const uint4 w = *reinterpret_cast<const uint4*>(kimg + swz_off(r, half * NCH + j));
+                k2[4 * j + 0] = bf2_to_f2(w.x);
+                k2[4 * j + 1] = bf2_to_f2(w.y);
+                k2[4 * j + 2] = bf2_to_f2(w.z);
+                k2[4 * j + 3] = bf2_to_f2(w.w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc = fma2(k2[4 * j + e], k2[4 * j + e], acc);
             }
+            sKn[half * 128 + r] = hsum2(acc);
         }
-        float kn = 0.f;
-#pragma unroll
-        for (int j = 0; j < D; ++j) kn = __fmaf_rn(k[j], k[j], kn);
 
         // issue the next tile's MMA into the other TMEM buffer (same head only)
         mma_issued_ahead = false;
@@ -283,82 +327,119 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             mma_issued_ahead = true;
         }
 
-        // ---- a1: nearest parent (expanded form from the tensor-core dots)
-        float best = INFINITY, second = INFINITY;
-        int bp = 0;
+        // ---- a1: this half's parents (16-column chunks c with c % 2 == half)
+        {
+            float best = INFINITY, second = INFINITY;
+            int bp = 0x7fffffff;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            if (16 * c < p.M0p) {
-                uint32_t r[16];
-                tmem_ld16(trow + 128 * s + 16 * c, r);
-                tmem_wait_ld();
-                tmem_touch16(r);
+            for (int cc = 0; cc < 4; ++cc) {
+                const int c = 2 * cc + half;
+                if (16 * c < p.M0p) {
+                    uint32_t v16[16];
+                    tmem_ld16(trow + 128 * s + 16 * c, v16);
+                    tmem_wait_ld();
+                    tmem_touch16(v16);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int pp = 16 * c + q;
-                    float dd = fmaf(-2.f, __uint_as_float(r[q]), kn + sCn[pp]);
-                    dd = pp < p.M0 ? dd : INFINITY;
-                    if (dd < best) { second = best; best = dd; bp = pp; }
-                    else second = fminf(second, dd);
+                    for (int q = 0; q < 16; q += 4) {
+                        const float4 cn4 = *reinterpret_cast<const float4*>(sCn + 16 * c + q);
+                        const float cnq[4] = {cn4.x, cn4.y, cn4.z, cn4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int pp = 16 * c + q + e;
+                            float v = fmaf(-2.f, __uint_as_float(v16[q + e]), cnq[e]);
+                            v = pp < p.M0 ? v : INFINITY;
+                            if (v < best) { second = best; best = v; bp = pp; }
+                            else second = fminf(second, v);
+                        }
+                    }
                 }
             }
+            sBest[half * 128 + r] = best;
+            sSecond[half * 128 + r] = second;
+            sIdx[half * 128 + r] = bp;
+        }
+        __syncthreads();
+        const float kn = sKn[r] + sKn[128 + r];
+        float best, second;
+        int bp;
+        {
+            const float b0 = sBest[r], b1 = sBest[128 + r];
+            const int i0 = sIdx[r], i1 = sIdx[128 + r];
+            const bool take1 = (b1 < b0) || (b1 == b0 && i1 < i0);
+            best = take1 ? b1 : b0;
+            bp = take1 ? i1 : i0;
+            second = fminf(fmaxf(b0, b1), fminf(sSecond[r], sSecond[128 + r]));
+            if (bp >= p.M0) bp = 0;   // no parent column (cannot happen for M0 >= 1)
         }
         const uint16_t* cbh = p.codebook + (size_t)h * p.Mtot * D;
+        const uint16_t* krow = p.K + ((size_t)bh * p.N + (size_t)t * kTile + r) * D;
         const float E = c_exp * (kn + cnmax);
         const bool redecide = valid && p.M0 > 1 && !(second - best > 2.f * E);
         if (__any_sync(0xffffffffu, redecide)) {
-            // re-decide among the parents within the band, in fp64; the TMEM
-            // reloads are warp-wide, the fp64 work only in the lanes that need it
+            // re-decide among the parents within the band, in fp64; both halves
+            // do it and reach the same result. TMEM reloads are warp-wide.
             double eb = INFINITY;
             int ep = bp;
             for (int c = 0; c < p.M0p; c += 16) {
-                uint32_t r[16];
-                tmem_ld16(trow + 128 * s + c, r);
+                uint32_t v16[16];
+                tmem_ld16(trow + 128 * s + c, v16);
                 tmem_wait_ld();
-                tmem_touch16(r);
+                tmem_touch16(v16);
                 if (redecide) {
                     for (int q = 0; q < 16; ++q) {
                         const int pp = c + q;
                         if (pp >= p.M0) break;
-                        const float dd = fmaf(-2.f, __uint_as_float(r[q]), kn + sCn[pp]);
-                        if (dd - best > 2.f * E) continue;
-                        const double e = exact_dist_reg<D>(k, cbh + (size_t)pp * D);
+                        const float v = fmaf(-2.f, __uint_as_float(v16[q]), sCn[pp]);
+                        if (v - best > 2.f * E) continue;
+                        const double e = exact_dist_glob<D>(krow, cbh + (size_t)pp * D);
                         if (e < eb) { eb = e; ep = pp; }
                     }
                 }
             }
             if (redecide) {
                 bp = ep;
-                ++n_pre;
+                if (half == 0) ++n_pre;
             }
         }
 
-        // ---- a2: the kept parent and its children, direct form
+        // ---- a2: partial direct distances of the kept parent and its children;
+        // half 1 publishes its partials, half 0 completes them and decides
+        float part[C + 1];
+        part[0] = half_dist<NCH>(k2, sB1, half * NCH, [&](int j) { return swz_off(bp, j); });
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            const int i = bp * C + c;
+            part[1 + c] = half_dist<NCH>(k2, sCh, half * NCH, [&](int j) { return ch_off<D>(i, bp, j); });
+        }
+        if (half == 1) {
+#pragma unroll
+            for (int c = 0; c <= C; ++c) sDist[c * 128 + r] = part[c];
+        }
+        __syncthreads();
         int leaf = bp;
-        {
-            const float dpar = direct_dist<D>(k, sB1 + 0, [&](int j) { return swz_off(bp, j); });
+        if (half == 0) {
+            const float dpar = __fadd_rn(part[0], sDist[r]);
             float dch[C];
             float lo = dpar;
             int lo_i = -1;
 #pragma unroll
             for (int c = 0; c < C; ++c) {
-                const int i = bp * C + c;
-                dch[c] = direct_dist<D>(k, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
+                dch[c] = __fadd_rn(part[1 + c], sDist[(1 + c) * 128 + r]);
                 if (dch[c] < lo) { lo = dch[c]; lo_i = c; }
             }
             bool sure = (lo_i < 0) || separated(lo, dpar, eps_dir);
 #pragma unroll
             for (int c = 0; c < C; ++c)
                 if (c != lo_i && !separated(lo, dch[c], eps_dir)) sure = false;
-            if (sure) {
+            if (sure || !valid) {
                 leaf = lo_i < 0 ? bp : p.M0 + bp * C + lo_i;
             } else {
-                double eb = exact_dist_reg<D>(k, cbh + (size_t)bp * D);
+                double eb = exact_dist_glob<D>(krow, cbh + (size_t)bp * D);
                 int win = bp;
 #pragma unroll
                 for (int c = 0; c < C; ++c) {
                     if (separated(lo, dch[c], eps_dir)) continue;
-                    const double e = exact_dist_reg<D>(k, cbh + (size_t)(p.M0 + bp * C + c) * D);
+                    const double e = exact_dist_glob<D>(krow, cbh + (size_t)(p.M0 + bp * C + c) * D);
                     if (e < eb) { eb = e; win = p.M0 + bp * C + c; }
                 }
                 leaf = win;
@@ -367,36 +448,37 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         }
 
         // ---- a3: outputs
-        if (tid < rows) {
-            p.assign[(size_t)bh * p.N + t * kTile + tid] = leaf;
-            atomicAdd(&sCnt[bp], 1);
-            if (leaf != bp) atomicAdd(&sCnt[leaf], 1);
+        if (half == 0) {
+            if (valid) {
+                p.assign[(size_t)bh * p.N + t * kTile + r] = leaf;
+                atomicAdd(&sCnt[bp], 1);
+                if (leaf != bp) atomicAdd(&sCnt[leaf], 1);
+            }
+            sPar[r] = valid ? bp : -1;
+            sLeaf[r] = leaf;
         }
-        sPar[tid] = tid < rows ? bp : -1;
-        sLeaf[tid] = leaf;
-        if (__syncthreads_or(!ok)) { failed = true; break; }   // also: K stage s free
+        if (__syncthreads_or(!ok)) { failed = true; break; }   // also: K stage s no longer read
 
-        // refill K stage s with tile g+2 (its V stage is refilled after the sums)
         const bool ok_v = mbar_wait(&bars[2 + s], (vph >> s) & 1u);
         vph ^= 1u << s;
         if (__syncthreads_or(!ok_v)) { failed = true; break; }
 
-        // value sums: warp w adds the V rows of keys 32w..32w+31
+        // value sums: warp w adds the V rows of keys 16w..16w+15
         {
             const uint8_t* vimg = sV0 + s * IMG;
             float* vs_bh = p.vsum + (size_t)bh * p.Mtot * D;
-            for (int q = 0; q < 32; ++q) {
-                const int r = 32 * warp + q;
-                const int par = sPar[r];
+            for (int q = 0; q < 16; ++q) {
+                const int rr = 16 * warp + q;
+                const int par = sPar[rr];
                 if (par < 0) break;
-                const int lf = sLeaf[r];
+                const int lf = sLeaf[rr];
                 if (D == 64) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(vimg + swz_off(r, lane >> 2) + (lane & 3) * 4);
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(vimg + swz_off(rr, lane >> 2) + (lane & 3) * 4);
                     const float a = bf_lo(w), b = bf_hi(w);
                     red_v2(vs_bh + (size_t)par * D + 2 * lane, a, b);
                     if (lf != par) red_v2(vs_bh + (size_t)lf * D + 2 * lane, a, b);
                 } else {
-                    const uint2 w = *reinterpret_cast<const uint2*>(vimg + swz_off(r, lane >> 1) + (lane & 1) * 8);
+                    const uint2 w = *reinterpret_cast<const uint2*>(vimg + swz_off(rr, lane >> 1) + (lane & 1) * 8);
                     const float a = bf_lo(w.x), b = bf_hi(w.x), c = bf_lo(w.y), d = bf_hi(w.y);
                     red_v4(vs_bh + (size_t)par * D + 4 * lane, a, b, c, d);
                     if (lf != par) red_v4(vs_bh + (size_t)lf * D + 4 * lane, a, b, c, d);
@@ -422,6 +504,12 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     }
 }
 
+size_t pre_smem_bytes(int D, int M0, int C, int Mtot) {
+    return 1024 + 5 * (size_t)(D / 64) * kRegion + (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) +
+           128 * 4 /*sCn*/ + 256 * 4 * 4 /*sKn, sBest, sSecond, sIdx*/ + (size_t)(C + 1) * 128 * 4 +
+           256 * 4 /*sPar, sLeaf*/ + 8 * 4 + (size_t)Mtot * 4 + 8 + 7 * 8 + 16;
+}
+
 template <int D, int C>
 cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, const void* cb, int32_t* assign,
                           int32_t* counts, float* vsum, StatusBlock* status, cudaStream_t st) {
@@ -441,14 +529,13 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     prm.Mtot = Mtot;
     prm.ntiles = (s.N + kTile - 1) / kTile;
     prm.total_tiles = prm.ntiles * BH;
+    prm.K = static_cast<const uint16_t*>(K);
     prm.codebook = static_cast<const uint16_t*>(cb);
     prm.assign = assign;
     prm.counts = counts;
     prm.vsum = vsum;
     prm.status = status;
-    const size_t ch_bytes = ((size_t)s.M0 * C * D * 2 + 15) & ~size_t(15);
-    const size_t smem = 1024 + 5 * (size_t)(D / 64) * kRegion + ch_bytes + 128 * 4 +
-                        (((size_t)Mtot + 3) & ~size_t(3)) * 4 + 256 * 4 + 16 + 8 + 7 * 8 + 16;
+    const size_t smem = pre_smem_bytes(D, s.M0, C, Mtot);
     auto kern = precompute_tc_kernel<D, C>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -456,25 +543,17 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = std::min(prm.total_tiles, sms);
-    kern<<<grid, 128, smem, st>>>(tk, tv, tcb, prm);
+    kern<<<grid, kThreads, smem, st>>>(tk, tv, tcb, prm);
     count_launch();
     return cudaGetLastError();
 }
 
 }  // namespace
 
-// Shared-memory bytes the tensor-core precompute needs (0 when it cannot run).
-size_t precompute_tc_smem(const avq_shape& s) {
-    const int D = s.d;
-    const size_t Mtot = (size_t)s.M0 * (1 + s.C);
-    return 1024 + 5 * (size_t)(D / 64) * kRegion + (((size_t)s.M0 * s.C * D * 2 + 15) & ~size_t(15)) +
-           128 * 4 + ((Mtot + 3) & ~size_t(3)) * 4 + 256 * 4 + 16 + 8 + 7 * 8 + 16;
-}
-
 bool precompute_tc_supported(const avq_shape& s) {
     if (s.dtype != AVQ_BF16 || (s.d != 64 && s.d != 128)) return false;
     if (!(s.C == 1 || s.C == 2 || s.C == 4 || s.C == 8 || s.C == 16)) return false;
-    return precompute_tc_smem(s) <= 227 * 1024;
+    return pre_smem_bytes(s.d, s.M0, s.C, s.M0 * (1 + s.C)) <= 227 * 1024;
 }
 
 cudaError_t launch_precompute_tc(const avq_shape& s, const void* K, const void* V, const void* cb,
