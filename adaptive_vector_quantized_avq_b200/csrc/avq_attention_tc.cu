@@ -232,7 +232,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         // ---- parent pass
         float x[128];
-        float m = -INFINITY;
+        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent partial maxima
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             // columns at or past M0p were not written by MMA1: never read them
@@ -259,11 +259,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 x[32 * c + k + 1] = fmaf(x[32 * c + k + 1], p.sl2, lb.y);
                 x[32 * c + k + 2] = fmaf(x[32 * c + k + 2], p.sl2, lb.z);
                 x[32 * c + k + 3] = fmaf(x[32 * c + k + 3], p.sl2, lb.w);
-                m = fmaxf(fmaxf(m, fmaxf(x[32 * c + k], x[32 * c + k + 1])),
-                          fmaxf(x[32 * c + k + 2], x[32 * c + k + 3]));
+                mp[(k >> 2) & 3] = fmaxf(mp[(k >> 2) & 3], fmaxf(fmaxf(x[32 * c + k], x[32 * c + k + 1]),
+                                                                 fmaxf(x[32 * c + k + 2], x[32 * c + k + 3])));
             }
         }
-        float z = 0.f;
+        const float m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        float zp[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             uint32_t w[8], e[16];
@@ -271,7 +272,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int k = 0; k < 16; ++k) {
                 const float ev = ex2(x[16 * c + k] - m);   // = A_p n_p (0 for empty parents)
                 x[16 * c + k] = ev;
-                z += ev;
+                zp[k & 3] += ev;
                 e[k] = __float_as_uint(ev);
             }
 #pragma unroll
@@ -279,6 +280,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_st8(trow + p.colW + 8 * c, w);   // bf16 weights: A operand of MMA3
             tmem_st16(trow + 16 * c, e);          // fp32 e'_p kept for the child pass
         }
+        const float z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
         // importance terms e'_p / Zbar_i (zero for rows past the end)
         const float rz = valid ? 1.f / z : 0.f;
 #pragma unroll
@@ -322,7 +324,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
 
         // ---- children, in chunks of <= 128 slots
-        float den = z;
+        float denp[4] = {z, 0.f, 0.f, 0.f};   // independent partial sums of the denominator
         const int PC = p.P * C;
         const int nchunks = (PC + kTile - 1) / kTile;
         for (int k = 0; k < nchunks; ++k) {
@@ -381,9 +383,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (__syncthreads_or(!ok)) { failed = true; break; }
             tc_fence_after();
 
-            // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m); denominator correction
+            // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m); denominator correction;
+            // only the 32-column groups that hold slots of this chunk
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
+                if (32 * c >= N2) break;
                 float sc[32];
                 tmem_ld32f(trow + p.colSc + 32 * c, sc);
                 uint32_t w[16];
@@ -398,7 +402,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         xmax = fmaxf(xmax, nc > 0.f ? xc : -INFINITY);
                         // slots past the chunk hold stale TMEM columns: their weight is 0
                         const float wc = nc > 0.f ? (ex2(xc) - ap[j / C]) * nc : 0.f;
-                        den += wc;
+                        denp[(kk >> 1) & 3] += wc;
                         dd[e] = wc;
                     }
                     w[kk / 2] = pack_bf16x2(dd[0], dd[1]);
@@ -429,7 +433,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
 
         // ---- epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
-        const float inv = 1.f / den;
+        const float inv = 1.f / ((denp[0] + denp[1]) + (denp[2] + denp[3]));
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             float o[32];

@@ -26,14 +26,14 @@
 //      error bound of this expanded form, the parents within the band are
 //      re-decided with the exact fp64 distance summed in index order.
 //   4. a2: the kept parent and its C children by the direct form
-//      sum_j (k_j - c_j)^2 in fp32 (packed f32x2 arithmetic, relative error
-//      <= (d+4)u); a candidate wins only when strictly closer (parent first,
+//      sum_j (k_j - c_j)^2 in fp32 (sm_100 mixed bf16/fp32 subtraction, so
+//      the codewords need no unpacking; relative error <= (d+4)u); a
+//      candidate wins only when strictly closer (parent first,
 //      lowest child index among equals); the band the bound cannot separate
 //      is re-decided in fp64.
 //   5. a3: assign written; counts in shared memory; the key's V row is added
 //      to the parent's and (when the key moved) the child's value sum with
-//      warp-wide coalesced fp32 vector reductions (one 256-byte row per
-//      instruction for d = 64).
+//      coalesced 16-byte fp32 vector reductions (one half-warp per row).
 #include <algorithm>
 
 #include "avq_internal.cuh"
@@ -77,50 +77,40 @@ __device__ __forceinline__ uint32_t ch_off(int i, int p, int j) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// packed fp32 pairs (sm_100 f32x2 arithmetic, round-to-nearest per lane)
-typedef unsigned long long f2_t;
-__device__ __forceinline__ f2_t pk2(float lo, float hi) {
-    f2_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+// (c - k) for a bf16 c (low or high half of a 32-bit word) and an fp32 k,
+// rounded once (sm_100 mixed-precision subtraction; no unpacking)
+__device__ __forceinline__ float sub_lo(uint32_t w, float k) {
+    float r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tsub.rn.f32.bf16 %0, l, %2;\n\t}" : "=f"(r) : "r"(w), "f"(k));
     return r;
 }
-__device__ __forceinline__ f2_t bf2_to_f2(uint32_t w) { return pk2(bf_lo(w), bf_hi(w)); }
-__device__ __forceinline__ f2_t sub2(f2_t a, f2_t b) {
-    f2_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+__device__ __forceinline__ float sub_hi(uint32_t w, float k) {
+    float r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tsub.rn.f32.bf16 %0, h, %2;\n\t}" : "=f"(r) : "r"(w), "f"(k));
     return r;
-}
-__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
-    f2_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-__device__ __forceinline__ float hsum2(f2_t a) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a));
-    return __fadd_rn(lo, hi);
 }
 
 // Partial squared distance over this half's NC 16-byte chunks (chunk index
-// offset j0) of the key (packed pairs) to a bf16 row in shared memory whose
-// chunk j lives at chunk_off(j); each term (k - c)^2 rounded once (fused).
+// offset j0) of the key (fp32) to a bf16 row in shared memory whose chunk j
+// lives at chunk_off(j); each term (k - c)^2 rounded once (fused), four
+// independent accumulators.
 template <int NC, typename F>
-__device__ __forceinline__ float half_dist(const f2_t (&k2)[NC * 4], const uint8_t* row_base, int j0,
+__device__ __forceinline__ float half_dist(const float (&k)[NC * 8], const uint8_t* row_base, int j0,
                                            F chunk_off) {
-    f2_t a = 0ull, b = 0ull;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
         const uint4 w = *reinterpret_cast<const uint4*>(row_base + chunk_off(j0 + j));
-        const f2_t t0 = sub2(k2[4 * j + 0], bf2_to_f2(w.x));
-        const f2_t t1 = sub2(k2[4 * j + 1], bf2_to_f2(w.y));
-        const f2_t t2 = sub2(k2[4 * j + 2], bf2_to_f2(w.z));
-        const f2_t t3 = sub2(k2[4 * j + 3], bf2_to_f2(w.w));
-        a = fma2(t0, t0, a);
-        b = fma2(t1, t1, b);
-        a = fma2(t2, t2, a);
-        b = fma2(t3, t3, b);
+        const float t0 = sub_lo(w.x, k[8 * j + 0]), t1 = sub_hi(w.x, k[8 * j + 1]);
+        const float t2 = sub_lo(w.y, k[8 * j + 2]), t3 = sub_hi(w.y, k[8 * j + 3]);
+        const float t4 = sub_lo(w.z, k[8 * j + 4]), t5 = sub_hi(w.z, k[8 * j + 5]);
+        const float t6 = sub_lo(w.w, k[8 * j + 6]), t7 = sub_hi(w.w, k[8 * j + 7]);
+        a0 = __fmaf_rn(t0, t0, a0); a1 = __fmaf_rn(t1, t1, a1);
+        a2 = __fmaf_rn(t2, t2, a2); a3 = __fmaf_rn(t3, t3, a3);
+        a0 = __fmaf_rn(t4, t4, a0); a1 = __fmaf_rn(t5, t5, a1);
+        a2 = __fmaf_rn(t6, t6, a2); a3 = __fmaf_rn(t7, t7, a3);
     }
-    return __fadd_rn(hsum2(a), hsum2(b));
+    return __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
 }
 
 // Exact fp64 distance between two global bf16 rows, terms in index order,
@@ -276,7 +266,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                         cn = __fmaf_rn(c, c, cn);
                     }
                 }
-                if (tid < 128) sCn[tid] = cn;
+                if (tid < 128) sCn[tid] = tid < p.M0 ? cn : INFINITY;
                 float mx = cn;
 #pragma unroll
                 for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -302,22 +292,25 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
 
-        // this half of the key row -> packed fp32 pairs; partial ||k||^2
-        f2_t k2[NCH * 4];
+        // this half of the key row -> fp32; partial ||k||^2
+        float k[NCH * 8];
         {
             const uint8_t* kimg = sK0 + s * IMG;
-            f2_t acc = 0ull;
+            float kn0 = 0.f, kn1 = 0.f;
 #pragma unroll
             for (int j = 0; j < NCH; ++j) {
                 const uint4 w = *reinterpret_cast<const uint4*>(kimg + swz_off(r, half * NCH + j));
-                k2[4 * j + 0] = bf2_to_f2(w.x);
-                k2[4 * j + 1] = bf2_to_f2(w.y);
-                k2[4 * j + 2] = bf2_to_f2(w.z);
-                k2[4 * j + 3] = bf2_to_f2(w.w);
+                k[8 * j + 0] = bf_lo(w.x); k[8 * j + 1] = bf_hi(w.x);
+                k[8 * j + 2] = bf_lo(w.y); k[8 * j + 3] = bf_hi(w.y);
+                k[8 * j + 4] = bf_lo(w.z); k[8 * j + 5] = bf_hi(w.z);
+                k[8 * j + 6] = bf_lo(w.w); k[8 * j + 7] = bf_hi(w.w);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc = fma2(k2[4 * j + e], k2[4 * j + e], acc);
+                for (int e = 0; e < 8; e += 2) {
+                    kn0 = __fmaf_rn(k[8 * j + e], k[8 * j + e], kn0);
+                    kn1 = __fmaf_rn(k[8 * j + e + 1], k[8 * j + e + 1], kn1);
+                }
             }
-            sKn[half * 128 + r] = hsum2(acc);
+            sKn[half * 128 + r] = __fadd_rn(kn0, kn1);
         }
 
         // issue the next tile's MMA into the other TMEM buffer (same head only)
@@ -327,10 +320,13 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             mma_issued_ahead = true;
         }
 
-        // ---- a1: this half's parents (16-column chunks c with c % 2 == half)
+        // ---- a1: this half's parents (16-column chunks c with c % 2 == half);
+        // four independent trackers over interleaved columns, merged at the end
         {
-            float best = INFINITY, second = INFINITY;
-            int bp = 0x7fffffff;
+            float best[4], second[4];
+            int bp[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) { best[u] = INFINITY; second[u] = INFINITY; bp[u] = 0x7fffffff; }
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 const int c = 2 * cc + half;
@@ -341,22 +337,31 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                     tmem_touch16(v16);
 #pragma unroll
                     for (int q = 0; q < 16; q += 4) {
+                        // ||C_p||^2 is +inf for padding parents (p >= M0)
                         const float4 cn4 = *reinterpret_cast<const float4*>(sCn + 16 * c + q);
                         const float cnq[4] = {cn4.x, cn4.y, cn4.z, cn4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int pp = 16 * c + q + e;
-                            float v = fmaf(-2.f, __uint_as_float(v16[q + e]), cnq[e]);
-                            v = pp < p.M0 ? v : INFINITY;
-                            if (v < best) { second = best; best = v; bp = pp; }
-                            else second = fminf(second, v);
+                        for (int u = 0; u < 4; ++u) {
+                            const int pp = 16 * c + q + u;
+                            const float v = fmaf(-2.f, __uint_as_float(v16[q + u]), cnq[u]);
+                            if (v < best[u]) { second[u] = best[u]; best[u] = v; bp[u] = pp; }
+                            else second[u] = fminf(second[u], v);
                         }
                     }
                 }
             }
-            sBest[half * 128 + r] = best;
-            sSecond[half * 128 + r] = second;
-            sIdx[half * 128 + r] = bp;
+            // merge the four trackers (lowest index among equal values)
+#pragma unroll
+            for (int u = 1; u < 4; ++u) {
+                const bool take = (best[u] < best[0]) || (best[u] == best[0] && bp[u] < bp[0]);
+                const float lo = take ? best[u] : best[0], hi = take ? best[0] : best[u];
+                second[0] = fminf(hi, fminf(second[0], second[u]));
+                best[0] = lo;
+                bp[0] = take ? bp[u] : bp[0];
+            }
+            sBest[half * 128 + r] = best[0];
+            sSecond[half * 128 + r] = second[0];
+            sIdx[half * 128 + r] = bp[0];
         }
         __syncthreads();
         const float kn = sKn[r] + sKn[128 + r];
@@ -405,11 +410,11 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         // ---- a2: partial direct distances of the kept parent and its children;
         // half 1 publishes its partials, half 0 completes them and decides
         float part[C + 1];
-        part[0] = half_dist<NCH>(k2, sB1, half * NCH, [&](int j) { return swz_off(bp, j); });
+        part[0] = half_dist<NCH>(k, sB1, half * NCH, [&](int j) { return swz_off(bp, j); });
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             const int i = bp * C + c;
-            part[1 + c] = half_dist<NCH>(k2, sCh, half * NCH, [&](int j) { return ch_off<D>(i, bp, j); });
+            part[1 + c] = half_dist<NCH>(k, sCh, half * NCH, [&](int j) { return ch_off<D>(i, bp, j); });
         }
         if (half == 1) {
 #pragma unroll
@@ -463,25 +468,37 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         vph ^= 1u << s;
         if (__syncthreads_or(!ok_v)) { failed = true; break; }
 
-        // value sums: warp w adds the V rows of keys 16w..16w+15
+        // value sums: warp w adds the V rows of keys 16w..16w+15, two keys per
+        // step (one per half-warp); lane l of a half holds 4 (d = 64) or 8
+        // (d = 128) consecutive dimensions of the row
         {
             const uint8_t* vimg = sV0 + s * IMG;
-            float* vs_bh = p.vsum + (size_t)bh * p.Mtot * D;
-            for (int q = 0; q < 16; ++q) {
-                const int rr = 16 * warp + q;
+            const int hl = lane & 15, sub = lane >> 4;
+            constexpr int DPL = D / 16;                       // dimensions per lane
+            const int j = (hl * DPL) >> 3;                    // 16-byte chunk of those dimensions
+            const uint32_t inchunk = ((hl * DPL) & 7) * 2;    // byte offset inside the chunk
+            float* vs_lane = p.vsum + (size_t)bh * p.Mtot * D + hl * DPL;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int rr = 16 * warp + 2 * q + sub;
                 const int par = sPar[rr];
-                if (par < 0) break;
                 const int lf = sLeaf[rr];
-                if (D == 64) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(vimg + swz_off(rr, lane >> 2) + (lane & 3) * 4);
-                    const float a = bf_lo(w), b = bf_hi(w);
-                    red_v2(vs_bh + (size_t)par * D + 2 * lane, a, b);
-                    if (lf != par) red_v2(vs_bh + (size_t)lf * D + 2 * lane, a, b);
-                } else {
-                    const uint2 w = *reinterpret_cast<const uint2*>(vimg + swz_off(rr, lane >> 1) + (lane & 1) * 8);
-                    const float a = bf_lo(w.x), b = bf_hi(w.x), c = bf_lo(w.y), d = bf_hi(w.y);
-                    red_v4(vs_bh + (size_t)par * D + 4 * lane, a, b, c, d);
-                    if (lf != par) red_v4(vs_bh + (size_t)lf * D + 4 * lane, a, b, c, d);
+                if (par >= 0) {
+                    const uint8_t* src = vimg + swz_off(rr, j) + inchunk;
+                    if (D == 64) {
+                        const uint2 w = *reinterpret_cast<const uint2*>(src);
+                        const float a = bf_lo(w.x), b = bf_hi(w.x), c = bf_lo(w.y), d = bf_hi(w.y);
+                        red_v4(vs_lane + (size_t)par * D, a, b, c, d);
+                        if (lf != par) red_v4(vs_lane + (size_t)lf * D, a, b, c, d);
+                    } else {
+                        const uint4 w = *reinterpret_cast<const uint4*>(src);
+                        red_v4(vs_lane + (size_t)par * D, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+                        red_v4(vs_lane + (size_t)par * D + 4, bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+                        if (lf != par) {
+                            red_v4(vs_lane + (size_t)lf * D, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+                            red_v4(vs_lane + (size_t)lf * D + 4, bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+                        }
+                    }
                 }
             }
         }

@@ -16,7 +16,6 @@ collective): weak scaling, value = all ranks' query rows / max-over-ranks time.
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import math
@@ -25,7 +24,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import numpy as np
@@ -223,21 +221,19 @@ def run_ours(args):
     import torch.distributed as dist
 
     from adaptive_vector_quantized_avq_b200 import binding as bd
+    from adaptive_vector_quantized_avq_b200 import multigpu as mg
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local, world = mg.env_rank_world()
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        mg.init("nccl", dev)
 
     wl = syn.WORKLOADS[args.workload]
     P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
-    wl_rank = wl.with_(seed=wl.seed + rank)
+    wl_rank = mg.rank_workload(wl, rank)
     inp = syn.generate(wl_rank)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
 
@@ -279,8 +275,7 @@ def run_ours(args):
             raise RuntimeError(f"avq call failed: {rc} {rc2}")
 
     def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
+        mg.barrier(dev)
 
     # warm-up
     for _ in range(args.warmup):
@@ -339,14 +334,11 @@ def run_ours(args):
     d2h = hO.numel() * hO.element_size()
 
     # max over ranks
-    vals = torch.tensor([ms_total, e2e_ms, statistics.mean(pre_ms), statistics.mean(att_ms)],
-                        device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms, pre_avg, att_avg = vals.tolist()
+    ms_total, e2e_ms, pre_avg, att_avg = mg.max_over_ranks(
+        [ms_total, e2e_ms, statistics.mean(pre_ms), statistics.mean(att_ms)], dev)
     ms_step = ms_total / args.steps
     rows_all = wl.rows * world
-    value = rows_all / (ms_step / 1e3)
+    value = mg.weak_scaling_value(wl.rows, world, ms_step)
 
     out = None
     if rank == 0:
@@ -379,7 +371,7 @@ def run_ours(args):
             "gpu_launches": int(launches),
         }
     if world > 1:
-        dist.barrier(device_ids=[local])
+        mg.barrier(dev)
         dist.destroy_process_group()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         smp = OracleSampler(wl, P)
@@ -422,6 +414,43 @@ def run_reference(args):
     }), flush=True)
 
 
+KERNEL_NAMES = {"precompute": "precompute_tc_kernel", "attention": "attention_tc_kernel"}
+
+
+def ingest_ncu(csv_path: str, workload: str, P: int):
+    """Record per-launch DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum)
+    of each kernel from an ncu --csv capture of this workload into
+    profiles/traffic.json, stamped with the current kernel-source hash."""
+    import csv
+    import collections
+    rows = list(csv.reader(open(csv_path)))
+    hdr = None
+    per = collections.defaultdict(lambda: collections.defaultdict(float))
+    for r in rows:
+        if r and r[0] == "ID":
+            hdr = r
+            continue
+        if hdr is None or len(r) != len(hdr):
+            continue
+        d = dict(zip(hdr, r))
+        name, metric, val, unit = d["Kernel Name"], d["Metric Name"], d["Metric Value"], d["Metric Unit"]
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1)
+        per[(d["ID"], name)][metric] = float(val.replace(",", "")) * scale
+    out = json.load(open(PROFILE_TRAFFIC)) if os.path.exists(PROFILE_TRAFFIC) else {}
+    for kind, kname in KERNEL_NAMES.items():
+        launches = [m for (i, n), m in per.items() if kname in n and "dram__bytes_read.sum" in m]
+        if not launches:
+            continue
+        b = [m["dram__bytes_read.sum"] + m.get("dram__bytes_write.sum", 0.0) for m in launches]
+        out[f"{kind}/{workload}/P{P}"] = {
+            "bytes_per_launch": sum(b) / len(b), "launches": len(b),
+            "source_hash": kernel_source_hash(kind), "from": os.path.basename(csv_path)}
+    os.makedirs(os.path.dirname(PROFILE_TRAFFIC), exist_ok=True)
+    with open(PROFILE_TRAFFIC, "w") as f:
+        json.dump(out, f, indent=1, sort_keys=True)
+    print(json.dumps(out, indent=1))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -432,7 +461,13 @@ def main(argv=None):
     ap.add_argument("--P", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--ingest-ncu", metavar="CSV", help="record DRAM traffic per launch from an ncu CSV")
     args = ap.parse_args(argv)
+    if args.ingest_ncu:
+        wl = syn.WORKLOADS[args.workload]
+        P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
+        ingest_ncu(args.ingest_ncu, args.workload, P)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
