@@ -107,28 +107,28 @@ __device__ __forceinline__ void butterfly_colsum64(float* v, int lane) {
 
 // 32 TMEM columns of this warp's lanes into v (one wait for both loads).
 __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* v) {
-    uint32_t a[16], b[16];
-    tmem_ld16(taddr, a);
-    tmem_ld16(taddr + 16, b);
+    tmem_ld16f(taddr, v);
+    tmem_ld16f(taddr + 16, v + 16);
     tmem_wait_ld();
-    tmem_touch16(a);
-    tmem_touch16(b);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        v[k] = __uint_as_float(a[k]);
-        v[16 + k] = __uint_as_float(b[k]);
-    }
+    tmem_touch16f(v);
+    tmem_touch16f(v + 16);
+}
+
+// pair barrier: the two warps (w and w+4) that share TMEM lanes 32w..32w+31
+__device__ __forceinline__ void pair_sync(int quarter) {
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
 }
 
 template <int D, int C, int MINB>
-__global__ void __launch_bounds__(128, MINB)
+__global__ void __launch_bounds__(256, MINB)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmCB, const __grid_constant__ CUtensorMap tmMN,
                     const TcAttnParams p) {
     constexpr int KH = D / 64;
     constexpr uint32_t IMG = KH * kRegion;           // bytes of one [128 x D] bf16 image
     constexpr int KSTEPS = D / 16;
-    constexpr int PAR_PER_CHUNK = kTile / C;         // selected parents covered by one child chunk
+    constexpr int PAR_PER_HALF = 64 / C;             // selected parents behind 64 child slots
+    constexpr int OD = D / 2;                        // output dimensions per half
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = align1024(smem_raw);
     uint8_t* const sQ0 = base;                       // two Q stages: sQ0, sQ0 + IMG
@@ -140,12 +140,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     float* sInvN = sLb + 128;                                // [128] 1 / n_p
     float* sNc = sInvN + 128;                                // [128] child counts of the chunk
     float* sPart = sNc + 128;                                // [4][128] importance partials
-    unsigned long long* sKey = reinterpret_cast<unsigned long long*>(sPart + 512);   // [128]
+    float* sX = sPart + 512;                                 // [2][128] row exchange (max, Zbar, den)
+    int* sRank = reinterpret_cast<int*>(sX + 256);           // [2][128] partial ranks
+    unsigned long long* sKey = reinterpret_cast<unsigned long long*>(sRank + 256);   // [128]
     int* sSel = reinterpret_cast<int*>(sKey + 128);          // [128] selected parents
     uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + 128);   // q0, q1, mma, head
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = tid & 127, hf = tid >> 7, quarter = warp & 3;
     const int g0 = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
     const int g1 = (int)(((long long)(blockIdx.x + 1) * p.total_tiles) / gridDim.x);
 
@@ -165,7 +168,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *sTmem;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's lane quarter
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);   // TMEM lanes of this row block
 
     const uint32_t idesc1 = idesc_bf16_f32(128, p.M0p, false);
     const uint32_t idesc3 = idesc_bf16_f32(128, D, true);
@@ -173,6 +176,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     float xmax = -INFINITY;
     bool failed = false;
     int cur_bh = -1;
+    const int c0 = 64 * hf;                     // this half's first parent column / child slot
 
     auto issue_q = [&](int g, int stage) {
         const int bh = g / p.ntiles, t = g % p.ntiles;
@@ -187,7 +191,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int stage = it & 1;
         const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
         const int rows = min(kTile, p.N - t * kTile);
-        const bool valid = tid < rows;
+        const bool valid = r < rows;
 
         // the previous tile's O store must have read the staging buffer (sB2)
         if (tid == 0) bulk_wait_read_all();
@@ -201,9 +205,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     tma_load_3d(sB3P + kh * kRegion, &tmMN, &bars[3], kh * 64, 0, bh);
                 }
             }
-            const int n = tid < p.M0 ? __ldg(p.counts + (size_t)bh * p.Mtot + tid) : 0;
-            sLb[tid] = n > 0 ? __log2f((float)n) : -INFINITY;
-            sInvN[tid] = n > 0 ? 1.f / (float)n : 0.f;
+            if (tid < 128) {
+                const int n = tid < p.M0 ? __ldg(p.counts + (size_t)bh * p.Mtot + tid) : 0;
+                sLb[tid] = n > 0 ? __log2f((float)n) : -INFINITY;
+                sInvN[tid] = n > 0 ? 1.f / (float)n : 0.f;
+            }
             const bool ok = mbar_wait(&bars[3], hphase);
             hphase ^= 1;
             if (__syncthreads_or(!ok)) { failed = true; break; }
@@ -230,43 +236,37 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
 
-        // ---- parent pass
-        float x[128];
-        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent partial maxima
+        // ---- parent pass over this half's 64 columns
+        float x[64];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            // columns at or past M0p were not written by MMA1: never read them
-            if (32 * c + 32 <= p.M0p) {
-                tmem_ld32f(trow + 32 * c, x + 32 * c);
-            } else if (32 * c + 16 <= p.M0p) {
-                uint32_t a[16];
-                tmem_ld16(trow + 32 * c, a);
-                tmem_wait_ld();
-                tmem_touch16(a);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    x[32 * c + k] = __uint_as_float(a[k]);
-                    x[32 * c + 16 + k] = -INFINITY;
-                }
+        for (int b = 0; b < 4; ++b) {   // columns at or past M0p were not written: never read them
+            if (c0 + 16 * b + 16 <= p.M0p) {
+                tmem_ld16f(trow + c0 + 16 * b, x + 16 * b);
             } else {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) x[32 * c + k] = -INFINITY;
-            }
-#pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-                const float4 lb = *reinterpret_cast<const float4*>(sLb + 32 * c + k);
-                x[32 * c + k + 0] = fmaf(x[32 * c + k + 0], p.sl2, lb.x);
-                x[32 * c + k + 1] = fmaf(x[32 * c + k + 1], p.sl2, lb.y);
-                x[32 * c + k + 2] = fmaf(x[32 * c + k + 2], p.sl2, lb.z);
-                x[32 * c + k + 3] = fmaf(x[32 * c + k + 3], p.sl2, lb.w);
-                mp[(k >> 2) & 3] = fmaxf(mp[(k >> 2) & 3], fmaxf(fmaxf(x[32 * c + k], x[32 * c + k + 1]),
-                                                                 fmaxf(x[32 * c + k + 2], x[32 * c + k + 3])));
+                for (int k = 0; k < 16; ++k) x[16 * b + k] = -INFINITY;
             }
         }
-        const float m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-        float zp[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int b = 0; b < 4; ++b) tmem_touch16f(x + 16 * b);
+        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int k = 0; k < 64; k += 4) {
+            const float4 lb = *reinterpret_cast<const float4*>(sLb + c0 + k);
+            x[k + 0] = fmaf(x[k + 0], p.sl2, lb.x);
+            x[k + 1] = fmaf(x[k + 1], p.sl2, lb.y);
+            x[k + 2] = fmaf(x[k + 2], p.sl2, lb.z);
+            x[k + 3] = fmaf(x[k + 3], p.sl2, lb.w);
+            mp[(k >> 2) & 3] = fmaxf(mp[(k >> 2) & 3], fmaxf(fmaxf(x[k], x[k + 1]), fmaxf(x[k + 2], x[k + 3])));
+        }
+        sX[hf * 128 + r] = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        pair_sync(quarter);
+        const float m = fmaxf(sX[r], sX[128 + r]);
+        pair_sync(quarter);
+        float zp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
             uint32_t w[8], e[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
@@ -277,37 +277,44 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) w[k] = pack_bf16x2(x[16 * c + 2 * k], x[16 * c + 2 * k + 1]);
-            tmem_st8(trow + p.colW + 8 * c, w);   // bf16 weights: A operand of MMA3
-            tmem_st16(trow + 16 * c, e);          // fp32 e'_p kept for the child pass
+            tmem_st8(trow + p.colW + (c0 >> 1) + 8 * c, w);   // bf16 weights: A operand of MMA3
+            tmem_st16(trow + c0 + 16 * c, e);                 // fp32 e'_p kept for the child pass
         }
-        const float z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
+        sX[hf * 128 + r] = (zp[0] + zp[1]) + (zp[2] + zp[3]);
+        pair_sync(quarter);
+        const float z = sX[r] + sX[128 + r];
         // importance terms e'_p / Zbar_i (zero for rows past the end)
         const float rz = valid ? 1.f / z : 0.f;
 #pragma unroll
-        for (int k = 0; k < 128; ++k) x[k] *= rz;
+        for (int k = 0; k < 64; ++k) x[k] *= rz;
         butterfly_colsum64(x, lane);
-        butterfly_colsum64(x + 64, lane);
-        reinterpret_cast<float2*>(sPart + warp * 128)[lane] = make_float2(x[0], x[1]);
-        reinterpret_cast<float2*>(sPart + warp * 128 + 64)[lane] = make_float2(x[64], x[65]);
+        reinterpret_cast<float2*>(sPart + quarter * 128 + c0)[lane] = make_float2(x[0], x[1]);
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
 
-        // ---- importance and top-P selection (rank over 64-bit keys)
+        // ---- importance and top-P selection: ranks over 64-bit keys, each
+        // thread of a pair counting over half of the parents
         {
-            const float w = (sPart[tid] + sPart[128 + tid]) + (sPart[256 + tid] + sPart[384 + tid]);
-            // larger importance first, then the lower index; w >= 0 so its bits order like its value
-            const unsigned long long key =
-                tid < p.M0 ? ((unsigned long long)__float_as_uint(w) << 32) | (uint32_t)(0xFFFFFFFFu - tid) : 0ull;
-            sKey[tid] = key;
+            if (tid < 128) {
+                const float w = (sPart[tid] + sPart[128 + tid]) + (sPart[256 + tid] + sPart[384 + tid]);
+                // larger importance first, then the lower index; w >= 0 orders like its bits
+                sKey[tid] = tid < p.M0 ? ((unsigned long long)__float_as_uint(w) << 32) |
+                                             (uint32_t)(0xFFFFFFFFu - tid)
+                                       : 0ull;
+            }
+            __syncthreads();
+            const unsigned long long key = sKey[r];
+            int rk = 0;
+#pragma unroll 8
+            for (int q = 0; q < 64; q += 2) {
+                const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(sKey + c0 + q);
+                rk += (kk.x > key) + (kk.y > key);
+            }
+            sRank[hf * 128 + r] = rk;
             __syncthreads();
             if (tid < p.M0) {
-                int rank = 0;
-#pragma unroll 8
-                for (int q = 0; q < 128; q += 2) {
-                    const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(sKey + q);
-                    rank += (kk.x > key) + (kk.y > key);
-                }
+                const int rank = sRank[tid] + sRank[128 + tid];
                 if (rank < p.P) {
                     sSel[rank] = tid;
                     p.selected[((size_t)bh * p.ntiles + t) * p.P + rank] = tid;
@@ -323,15 +330,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 mma_ts(tmem + p.colO, tmem + p.colW + 8 * ks, desc_mn(sB3P, ks), idesc3, ks > 0);
         }
 
-        // ---- children, in chunks of <= 128 slots
-        float denp[4] = {z, 0.f, 0.f, 0.f};   // independent partial sums of the denominator
+        // ---- children, in chunks of <= 128 slots (this half: slots 64hf..64hf+63)
+        float denp[4] = {0.f, 0.f, 0.f, 0.f};   // child corrections of the denominator
         const int PC = p.P * C;
         const int nchunks = (PC + kTile - 1) / kTile;
         for (int k = 0; k < nchunks; ++k) {
             const int s0 = k * kTile;
             const int ns = min(kTile, PC - s0);
             const int N2 = (ns + 15) & ~15;
-            for (int idx = tid; idx < N2 * (D / 8); idx += 128) {
+            for (int idx = tid; idx < N2 * (D / 8); idx += 256) {
                 const int slot = idx / (D / 8), j = idx % (D / 8);
                 const uint32_t off = swz(slot, j);
                 if (slot < ns) {
@@ -345,7 +352,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
             }
             cp_async_commit();
-            {
+            if (tid < 128) {
                 float nc = 0.f;
                 if (tid < ns) {
                     const int sg = s0 + tid;
@@ -353,17 +360,18 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 sNc[tid] = nc;
             }
-            // A_p = e'_p / n_p of the chunk's parents, read before MMA2 may reuse the columns
-            float ap[PAR_PER_CHUNK];
+            // A_p = e'_p / n_p of this half's parents, read before MMA2 may reuse the columns
+            float ap[PAR_PER_HALF];
             {
-                uint32_t r[PAR_PER_CHUNK];
+                const int q0 = (s0 + c0) / C;
+                uint32_t rr[PAR_PER_HALF];
 #pragma unroll
-                for (int q = 0; q < PAR_PER_CHUNK; ++q) tmem_ld1(trow + sSel[min(s0 / C + q, p.P - 1)], r[q]);
+                for (int q = 0; q < PAR_PER_HALF; ++q) tmem_ld1(trow + sSel[min(q0 + q, p.P - 1)], rr[q]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < PAR_PER_CHUNK; ++q) {
-                    tmem_touch1(r[q]);
-                    ap[q] = __uint_as_float(r[q]) * sInvN[sSel[min(s0 / C + q, p.P - 1)]];
+                for (int q = 0; q < PAR_PER_HALF; ++q) {
+                    tmem_touch1(rr[q]);
+                    ap[q] = __uint_as_float(rr[q]) * sInvN[sSel[min(q0 + q, p.P - 1)]];
                 }
             }
             cp_async_wait_all();
@@ -383,21 +391,20 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (__syncthreads_or(!ok)) { failed = true; break; }
             tc_fence_after();
 
-            // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m); denominator correction;
-            // only the 32-column groups that hold slots of this chunk
+            // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m) for this half's slots
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (32 * c >= N2) break;
+            for (int c = 0; c < 2; ++c) {
+                if (c0 + 32 * c >= N2) break;
                 float sc[32];
-                tmem_ld32f(trow + p.colSc + 32 * c, sc);
+                tmem_ld32f(trow + p.colSc + c0 + 32 * c, sc);
                 uint32_t w[16];
 #pragma unroll
                 for (int kk = 0; kk < 32; kk += 2) {
                     float dd[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int j = 32 * c + kk + e;
-                        const float nc = sNc[j];
+                        const int j = 32 * c + kk + e;            // slot within this half
+                        const float nc = sNc[c0 + j];
                         const float xc = fminf(fmaf(sc[kk + e], p.sl2, -m), 126.f);
                         xmax = fmaxf(xmax, nc > 0.f ? xc : -INFINITY);
                         // slots past the chunk hold stale TMEM columns: their weight is 0
@@ -407,7 +414,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     }
                     w[kk / 2] = pack_bf16x2(dd[0], dd[1]);
                 }
-                tmem_st16(trow + p.colWc + 16 * c, w);
+                tmem_st16(trow + p.colWc + (c0 >> 1) + 16 * c, w);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -433,11 +440,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
 
         // ---- epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
-        const float inv = 1.f / ((denp[0] + denp[1]) + (denp[2] + denp[3]));
+        sX[hf * 128 + r] = (denp[0] + denp[1]) + (denp[2] + denp[3]);
+        pair_sync(quarter);
+        const float inv = 1.f / (z + (sX[r] + sX[128 + r]));
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < OD / 32; ++c) {
             float o[32];
-            tmem_ld32f(trow + p.colO + 32 * c, o);
+            tmem_ld32f(trow + p.colO + hf * OD + 32 * c, o);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint4 u;
@@ -445,7 +454,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 u.y = pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
                 u.z = pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
                 u.w = pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-                *reinterpret_cast<uint4*>(sB2 + swz(tid, 4 * c + q)) = u;
+                *reinterpret_cast<uint4*>(sB2 + swz(r, hf * (OD / 8) + 4 * c + q)) = u;
             }
         }
         fence_proxy_async_smem();
@@ -522,7 +531,7 @@ cudaError_t launch_tc(const avq_shape& s, const void* Q, const void* cb, const i
     prm.means = static_cast<const uint16_t*>(means);
     prm.selected = selected;
     prm.status = status;
-    const size_t need = 1024 + 6 * (size_t)(D / 64) * kRegion + 4096 + 1024 + 64;
+    const size_t need = 1024 + 6 * (size_t)(D / 64) * kRegion + 8192 + 64;
     // with 512 TMEM columns per CTA at most one CTA may be resident per SM:
     // then ask for more than half of the SM's shared memory
     const size_t smem = MINB == 2 ? need : std::max<size_t>(need, 120 * 1024);
@@ -533,7 +542,7 @@ cudaError_t launch_tc(const avq_shape& s, const void* Q, const void* cb, const i
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = std::min(prm.total_tiles, sms * MINB);
-    kern<<<grid, 128, smem, st>>>(tq, to, tcb, tmn, prm);
+    kern<<<grid, 256, smem, st>>>(tq, to, tcb, tmn, prm);
     count_launch();
     return cudaGetLastError();
 }
