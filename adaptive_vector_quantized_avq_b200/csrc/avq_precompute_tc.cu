@@ -61,13 +61,15 @@ struct TcPreParams {
 __device__ __forceinline__ uint8_t* align1024p(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
-__device__ __forceinline__ uint64_t desc_k128(const uint8_t* img, int ks) {
-    const uint32_t a = smem_u32(img) + (uint32_t)(ks >> 2) * kRegion + (uint32_t)(ks & 3) * 32u;
+// K-major operand, k-step ks, of a [rows x D] bf16 image whose 64-column
+// blocks are `region` bytes apart
+__device__ __forceinline__ uint64_t desc_k128(const uint8_t* img, int ks, uint32_t region = kRegion) {
+    const uint32_t a = smem_u32(img) + (uint32_t)(ks >> 2) * region + (uint32_t)(ks & 3) * 32u;
     return smem_desc_sw128(a, 16, 1024);
 }
 // 16-byte chunk j of row r of a TMA 128-byte-swizzled [rows x D] image
-__device__ __forceinline__ uint32_t swz_off(int r, int j) {
-    return (uint32_t)(j >> 3) * kRegion + (uint32_t)r * 128u + (uint32_t)(((j & 7) ^ (r & 7)) << 4);
+__device__ __forceinline__ uint32_t swz_off(int r, int j, uint32_t region = kRegion) {
+    return (uint32_t)(j >> 3) * region + (uint32_t)r * 128u + (uint32_t)(((j & 7) ^ (r & 7)) << 4);
 }
 // 16-byte chunk j of child row i (parent p = i / C) in the children image
 template <int D>
@@ -135,7 +137,7 @@ __device__ __forceinline__ void red_v4(float* addr, float a, float b, float c, f
                  : "memory");
 }
 
-template <int D, int C>
+template <int D, int C, int KVS>
 __global__ void __launch_bounds__(kThreads, 1)
 precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmCB, const TcPreParams p) {
@@ -145,10 +147,11 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     constexpr int NCH = D / 16;          // 16-byte chunks per half row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = align1024p(smem_raw);
-    uint8_t* sK0 = base;                     // K stages: sK0 + s*IMG
-    uint8_t* sV0 = base + 2 * IMG;           // V stages
-    uint8_t* sB1 = base + 4 * IMG;           // parent codewords (K-major, TMA)
-    uint8_t* sCh = base + 5 * IMG;           // children image [M0*C rows x D] bf16
+    uint8_t* sK0 = base;                     // K stages: sK0 + s*IMG (KVS of them)
+    uint8_t* sV0 = base + KVS * IMG;         // V stages
+    uint8_t* sB1 = base + 2 * KVS * IMG;     // parent codewords (K-major, TMA), M0p rows
+    const uint32_t b1_region = (uint32_t)p.M0p * 128u;   // bytes between its 64-column blocks
+    uint8_t* sCh = sB1 + KH * b1_region;     // children image [M0*C rows x D] bf16
     const size_t ch_bytes = (size_t)p.M0 * C * D * 2;
     float* sCn = reinterpret_cast<float*>(sCh + ((ch_bytes + 15) & ~size_t(15)));   // [128]
     float* sKn = sCn + 128;                  // [2][128] partial ||k||^2
@@ -199,7 +202,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     float cnmax = 0.f;
     int n_pre = 0, n_chd = 0;   // fp64 re-decisions (diagnostics)
 
-    auto issue_kv = [&](int g, int s) {
+    auto issue_kv = [&](int g, int s) {   // K and V tiles of tile g into stage s
         const int bh = g / p.ntiles, t = g % p.ntiles;
         mbar_arrive_expect_tx(&bars[s], IMG);
         mbar_arrive_expect_tx(&bars[2 + s], IMG);
@@ -209,15 +212,15 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             tma_load_3d(sV0 + s * IMG + kh * kRegion, &tmV, &bars[2 + s], kh * 64, t * kTile, bh);
         }
     };
-    auto issue_mma = [&](int s) -> bool {   // tid 0 only
+    auto issue_mma = [&](int s, int tb) -> bool {   // tid 0 only: K stage s -> TMEM buffer tb
         const bool ok = mbar_wait(&bars[s], (kph >> s) & 1u);
         kph ^= 1u << s;
         if (!ok) return false;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks)
-            mma_ss(tmem + 128 * s, desc_k128(sK0 + s * IMG, ks), desc_k128(sB1, ks), idesc, ks > 0);
-        mma_commit(&bars[4 + s]);
+            mma_ss(tmem + 128 * tb, desc_k128(sK0 + s * IMG, ks), desc_k128(sB1, ks, b1_region), idesc, ks > 0);
+        mma_commit(&bars[4 + tb]);
         return true;
     };
     auto flush_counts = [&](int bh) {
@@ -232,12 +235,13 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 
     if (tid == 0 && g0 < g1) {
         issue_kv(g0, 0);
-        if (g0 + 1 < g1) issue_kv(g0 + 1, 1);
+        if (KVS == 2 && g0 + 1 < g1) issue_kv(g0 + 1, 1);
     }
     bool mma_issued_ahead = false;   // MMA of the current tile already issued
 
     for (int g = g0, it = 0; g < g1; ++g, ++it) {
-        const int s = it & 1;
+        const int s = KVS == 2 ? (it & 1) : 0;   // K/V stage
+        const int tb = it & 1;                   // TMEM buffer of this tile's dot products
         const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
         const int rows = min(kTile, p.N - t * kTile);
         const bool valid = r < rows;
@@ -249,7 +253,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                 if (tid == 0) {
                     mbar_arrive_expect_tx(&bars[6], KH * (uint32_t)p.M0p * 128u);
 #pragma unroll
-                    for (int kh = 0; kh < KH; ++kh) tma_load_3d(sB1 + kh * kRegion, &tmCB, &bars[6], kh * 64, 0, h);
+                    for (int kh = 0; kh < KH; ++kh) tma_load_3d(sB1 + kh * b1_region, &tmCB, &bars[6], kh * 64, 0, h);
                 }
                 const uint16_t* chg = p.codebook + ((size_t)h * p.Mtot + p.M0) * D;
                 for (int idx = tid; idx < p.M0 * C * (D / 8); idx += kThreads) {
@@ -285,10 +289,10 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         }
 
         bool ok = true;
-        if (tid == 0 && !mma_issued_ahead) ok = issue_mma(s);
+        if (tid == 0 && !mma_issued_ahead) ok = issue_mma(s, tb);
         if (__syncthreads_or(!ok)) { failed = true; break; }
-        ok = mbar_wait(&bars[4 + s], (mph >> s) & 1u);
-        mph ^= 1u << s;
+        ok = mbar_wait(&bars[4 + tb], (mph >> tb) & 1u);
+        mph ^= 1u << tb;
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
 
@@ -313,10 +317,11 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             sKn[half * 128 + r] = __fadd_rn(kn0, kn1);
         }
 
-        // issue the next tile's MMA into the other TMEM buffer (same head only)
+        // issue the next tile's MMA into the other TMEM buffer (same head, and
+        // only when its K tile is already on the way: two K/V stages)
         mma_issued_ahead = false;
-        if (g + 1 < g1 && (g + 1) / p.ntiles == bh) {
-            if (tid == 0) ok = issue_mma(s ^ 1);
+        if (KVS == 2 && g + 1 < g1 && (g + 1) / p.ntiles == bh) {
+            if (tid == 0) ok = issue_mma(s ^ 1, tb ^ 1);
             mma_issued_ahead = true;
         }
 
@@ -332,7 +337,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                 const int c = 2 * cc + half;
                 if (16 * c < p.M0p) {
                     uint32_t v16[16];
-                    tmem_ld16(trow + 128 * s + 16 * c, v16);
+                    tmem_ld16(trow + 128 * tb + 16 * c, v16);
                     tmem_wait_ld();
                     tmem_touch16(v16);
 #pragma unroll
@@ -387,7 +392,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             int ep = bp;
             for (int c = 0; c < p.M0p; c += 16) {
                 uint32_t v16[16];
-                tmem_ld16(trow + 128 * s + c, v16);
+                tmem_ld16(trow + 128 * tb + c, v16);
                 tmem_wait_ld();
                 tmem_touch16(v16);
                 if (redecide) {
@@ -410,7 +415,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         // ---- a2: partial direct distances of the kept parent and its children;
         // half 1 publishes its partials, half 0 completes them and decides
         float part[C + 1];
-        part[0] = half_dist<NCH>(k, sB1, half * NCH, [&](int j) { return swz_off(bp, j); });
+        part[0] = half_dist<NCH>(k, sB1, half * NCH, [&](int j) { return swz_off(bp, j, b1_region); });
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             const int i = bp * C + c;
@@ -503,7 +508,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             }
         }
         __syncthreads();
-        if (tid == 0 && g + 2 < g1) issue_kv(g + 2, s);
+        if (tid == 0 && g + KVS < g1) issue_kv(g + KVS, s);
     }
 
     if (!failed && cur_bh >= 0) flush_counts(cur_bh);
@@ -522,9 +527,12 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 }
 
 size_t pre_smem_bytes(int D, int M0, int C, int Mtot) {
-    return 1024 + 5 * (size_t)(D / 64) * kRegion + (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) +
-           128 * 4 /*sCn*/ + 256 * 4 * 4 /*sKn, sBest, sSecond, sIdx*/ + (size_t)(C + 1) * 128 * 4 +
-           256 * 4 /*sPar, sLeaf*/ + 8 * 4 + (size_t)Mtot * 4 + 8 + 7 * 8 + 16;
+    const int kvs = D == 64 ? 2 : 1;
+    const size_t M0p = (size_t)((M0 + 15) & ~15);
+    return 1024 + 2 * kvs * (size_t)(D / 64) * kRegion + (size_t)(D / 64) * M0p * 128 +
+           (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) + 128 * 4 /*sCn*/ +
+           256 * 4 * 4 /*sKn, sBest, sSecond, sIdx*/ + (size_t)(C + 1) * 128 * 4 + 256 * 4 /*sPar, sLeaf*/ +
+           8 * 4 + (size_t)Mtot * 4 + 8 + 7 * 8 + 16;
 }
 
 template <int D, int C>
@@ -553,7 +561,7 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     prm.vsum = vsum;
     prm.status = status;
     const size_t smem = pre_smem_bytes(D, s.M0, C, Mtot);
-    auto kern = precompute_tc_kernel<D, C>;
+    auto kern = precompute_tc_kernel<D, C, D == 64 ? 2 : 1>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
