@@ -127,7 +127,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     constexpr int KH = D / 64;
     constexpr uint32_t IMG = KH * kRegion;           // bytes of one [128 x D] bf16 image
     constexpr int KSTEPS = D / 16;
-    constexpr int PAR_PER_HALF = 64 / C;             // selected parents behind 64 child slots
+    constexpr int PPB = 32 / C;                      // selected parents behind a 32-slot block
     constexpr int OD = D / 2;                        // output dimensions per half
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = align1024(smem_raw);
@@ -176,7 +176,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     float xmax = -INFINITY;
     bool failed = false;
     int cur_bh = -1;
-    const int c0 = 64 * hf;                     // this half's first parent column / child slot
+    // Work split of a row between its two threads: half hf owns the 16-column
+    // parent blocks 2b+hf (columns 32b+16hf..+16) and the 32-slot child blocks
+    // 2c+hf (slots 64c+32hf..+32), so both halves stay busy for any M0 and P*C.
+    const int c0 = 64 * hf;                     // this half's keys in the rank count
 
     auto issue_q = [&](int g, int stage) {
         const int bh = g / p.ntiles, t = g % p.ntiles;
@@ -230,8 +233,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (g + 1 < g1) issue_q(g + 1, stage ^ 1);
             }
         }
-        if (__syncthreads_or(!ok)) { failed = true; break; }
-        ok = mbar_wait(&bars[2], mphase);
+        // (if thread 0 could not issue MMA1, every thread's wait below times out)
+        ok = mbar_wait(&bars[2], mphase) && ok;
         mphase ^= 1;
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
@@ -240,8 +243,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         float x[64];
 #pragma unroll
         for (int b = 0; b < 4; ++b) {   // columns at or past M0p were not written: never read them
-            if (c0 + 16 * b + 16 <= p.M0p) {
-                tmem_ld16f(trow + c0 + 16 * b, x + 16 * b);
+            if (32 * b + 16 * hf + 16 <= p.M0p) {
+                tmem_ld16f(trow + 32 * b + 16 * hf, x + 16 * b);
             } else {
 #pragma unroll
                 for (int k = 0; k < 16; ++k) x[16 * b + k] = -INFINITY;
@@ -253,7 +256,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int k = 0; k < 64; k += 4) {
-            const float4 lb = *reinterpret_cast<const float4*>(sLb + c0 + k);
+            const float4 lb = *reinterpret_cast<const float4*>(sLb + 32 * (k >> 4) + 16 * hf + (k & 15));
             x[k + 0] = fmaf(x[k + 0], p.sl2, lb.x);
             x[k + 1] = fmaf(x[k + 1], p.sl2, lb.y);
             x[k + 2] = fmaf(x[k + 2], p.sl2, lb.z);
@@ -277,8 +280,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) w[k] = pack_bf16x2(x[16 * c + 2 * k], x[16 * c + 2 * k + 1]);
-            tmem_st8(trow + p.colW + (c0 >> 1) + 8 * c, w);   // bf16 weights: A operand of MMA3
-            tmem_st16(trow + c0 + 16 * c, e);                 // fp32 e'_p kept for the child pass
+            tmem_st8(trow + p.colW + 16 * c + 8 * hf, w);     // bf16 weights: A operand of MMA3
+            tmem_st16(trow + 32 * c + 16 * hf, e);            // fp32 e'_p kept for the child pass
         }
         sX[hf * 128 + r] = (zp[0] + zp[1]) + (zp[2] + zp[3]);
         pair_sync(quarter);
@@ -288,7 +291,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
         for (int k = 0; k < 64; ++k) x[k] *= rz;
         butterfly_colsum64(x, lane);
-        reinterpret_cast<float2*>(sPart + quarter * 128 + c0)[lane] = make_float2(x[0], x[1]);
+        // lane L now holds the row-block sums of this half's x[2L], x[2L+1], i.e.
+        // of parent columns 32(L/8) + 16hf + 2(L%8) and the next one
+        *reinterpret_cast<float2*>(sPart + quarter * 128 + 32 * (lane >> 3) + 16 * hf + 2 * (lane & 7)) =
+            make_float2(x[0], x[1]);
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
@@ -360,19 +366,25 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 sNc[tid] = nc;
             }
-            // A_p = e'_p / n_p of this half's parents, read before MMA2 may reuse the columns
-            float ap[PAR_PER_HALF];
+            // A_p = e'_p / n_p of the parents behind this half's two slot blocks,
+            // read before MMA2 may reuse the columns
+            float ap[2][PPB];
             {
-                const int q0 = (s0 + c0) / C;
-                uint32_t rr[PAR_PER_HALF];
+                uint32_t rr[2][PPB];
 #pragma unroll
-                for (int q = 0; q < PAR_PER_HALF; ++q) tmem_ld1(trow + sSel[min(q0 + q, p.P - 1)], rr[q]);
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int q = 0; q < PPB; ++q)
+                        tmem_ld1(trow + sSel[min((s0 + 64 * c + 32 * hf) / C + q, p.P - 1)], rr[c][q]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < PAR_PER_HALF; ++q) {
-                    tmem_touch1(rr[q]);
-                    ap[q] = __uint_as_float(rr[q]) * sInvN[sSel[min(q0 + q, p.P - 1)]];
-                }
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int q = 0; q < PPB; ++q) {
+                        tmem_touch1(rr[c][q]);
+                        ap[c][q] = __uint_as_float(rr[c][q]) *
+                                   sInvN[sSel[min((s0 + 64 * c + 32 * hf) / C + q, p.P - 1)]];
+                    }
             }
             cp_async_wait_all();
             fence_proxy_async_smem();
@@ -394,27 +406,28 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m) for this half's slots
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                if (c0 + 32 * c >= N2) break;
+                const int sb = 64 * c + 32 * hf;                   // first slot of this block
+                if (sb >= N2) break;
                 float sc[32];
-                tmem_ld32f(trow + p.colSc + c0 + 32 * c, sc);
+                tmem_ld32f(trow + p.colSc + sb, sc);
                 uint32_t w[16];
 #pragma unroll
                 for (int kk = 0; kk < 32; kk += 2) {
                     float dd[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int j = 32 * c + kk + e;            // slot within this half
-                        const float nc = sNc[c0 + j];
+                        const int j = kk + e;                      // slot within the block
+                        const float nc = sNc[sb + j];
                         const float xc = fminf(fmaf(sc[kk + e], p.sl2, -m), 126.f);
                         xmax = fmaxf(xmax, nc > 0.f ? xc : -INFINITY);
                         // slots past the chunk hold stale TMEM columns: their weight is 0
-                        const float wc = nc > 0.f ? (ex2(xc) - ap[j / C]) * nc : 0.f;
+                        const float wc = nc > 0.f ? (ex2(xc) - ap[c][j / C]) * nc : 0.f;
                         denp[(kk >> 1) & 3] += wc;
                         dd[e] = wc;
                     }
                     w[kk / 2] = pack_bf16x2(dd[0], dd[1]);
                 }
-                tmem_st16(trow + p.colWc + (c0 >> 1) + 16 * c, w);
+                tmem_st16(trow + p.colWc + (sb >> 1), w);
             }
             tmem_wait_st();
             tc_fence_before();

@@ -290,8 +290,8 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 
         bool ok = true;
         if (tid == 0 && !mma_issued_ahead) ok = issue_mma(s, tb);
-        if (__syncthreads_or(!ok)) { failed = true; break; }
-        ok = mbar_wait(&bars[4 + tb], (mph >> tb) & 1u);
+        // (if thread 0 could not issue the MMA, every thread's wait below times out)
+        ok = mbar_wait(&bars[4 + tb], (mph >> tb) & 1u) && ok;
         mph ^= 1u << tb;
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
@@ -467,11 +467,9 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             sPar[r] = valid ? bp : -1;
             sLeaf[r] = leaf;
         }
-        if (__syncthreads_or(!ok)) { failed = true; break; }   // also: K stage s no longer read
-
         const bool ok_v = mbar_wait(&bars[2 + s], (vph >> s) & 1u);
         vph ^= 1u << s;
-        if (__syncthreads_or(!ok_v)) { failed = true; break; }
+        if (__syncthreads_or(!ok || !ok_v)) { failed = true; break; }   // also: K stage s no longer read
 
         // value sums: warp w adds the V rows of keys 16w..16w+15, two keys per
         // step (one per half-warp); lane l of a half holds 4 (d = 64) or 8
