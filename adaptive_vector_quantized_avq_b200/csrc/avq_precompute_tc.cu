@@ -45,12 +45,12 @@ using namespace sm100;
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 256;
 constexpr uint32_t kRegion = 128 * 128;
 
 struct TcPreParams {
     int BH, H, N, M0, M0p, Mtot, ntiles, total_tiles;
     const uint16_t* K;          // [BH, N, D] bf16 (exact re-decisions read keys here)
+    const uint16_t* V;          // [BH, N, D] bf16
     const uint16_t* codebook;   // [H, Mtot, D] bf16
     int32_t* assign;            // [BH, N]
     int32_t* counts;            // [BH, Mtot]
@@ -92,23 +92,51 @@ __device__ __forceinline__ float sub_hi(uint32_t w, float k) {
     return r;
 }
 
-// Exact fp64 distance between two global bf16 rows, terms in index order,
-// no fused operations.
-template <int D>
-__device__ __noinline__ double exact_dist_glob(const uint16_t* k, const uint16_t* c) {
+// Exact fp64 squared distance between two bf16 rows held in shared memory
+// (16-byte chunk j of each at xoff(j) / coff(j) from its base): terms
+// (x_j - c_j)^2 in index order, no fused operations, so that the sum is the
+// same double as a plain sequential fp64 loop over the row.
+template <int D, typename FX, typename FC>
+__device__ __noinline__ double exact_dist_smem(const uint8_t* xbase, FX xoff, const uint8_t* cbase, FC coff) {
     double s = 0.0;
-    for (int j = 0; j < D; ++j) {
-        const double kj = (double)__uint_as_float((uint32_t)__ldg(k + j) << 16);
-        const double cj = (double)__uint_as_float((uint32_t)__ldg(c + j) << 16);
-        const double t = __dsub_rn(kj, cj);
-        s = __dadd_rn(s, __dmul_rn(t, t));
+#pragma unroll 1
+    for (int j = 0; j < D / 8; ++j) {
+        const uint4 xw = *reinterpret_cast<const uint4*>(xbase + xoff(j));
+        const uint4 cw = *reinterpret_cast<const uint4*>(cbase + coff(j));
+        const uint32_t xs[4] = {xw.x, xw.y, xw.z, xw.w}, cs[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double x = (double)((e & 1) ? bf_hi(xs[e >> 1]) : bf_lo(xs[e >> 1]));
+            const double c = (double)((e & 1) ? bf_hi(cs[e >> 1]) : bf_lo(cs[e >> 1]));
+            const double t = __dsub_rn(x, c);
+            s = __dadd_rn(s, __dmul_rn(t, t));
+        }
+    }
+    return s;
+}
+// The same with the key's bf16 row in global memory (read once, all chunks
+// in flight together).
+template <int D, typename FC>
+__device__ __noinline__ double exact_dist_gk(const uint16_t* krow, const uint8_t* cbase, FC coff) {
+    uint4 kw[D / 8];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) kw[j] = __ldg(reinterpret_cast<const uint4*>(krow) + j);
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+        const uint4 cw = *reinterpret_cast<const uint4*>(cbase + coff(j));
+        const uint32_t xs[4] = {kw[j].x, kw[j].y, kw[j].z, kw[j].w}, cs[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double x = (double)((e & 1) ? bf_hi(xs[e >> 1]) : bf_lo(xs[e >> 1]));
+            const double c = (double)((e & 1) ? bf_hi(cs[e >> 1]) : bf_lo(cs[e >> 1]));
+            const double t = __dsub_rn(x, c);
+            s = __dadd_rn(s, __dmul_rn(t, t));
+        }
     }
     return s;
 }
 
-__device__ __forceinline__ void red_v2(float* addr, float a, float b) {
-    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
-}
 __device__ __forceinline__ void red_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
@@ -151,62 +179,73 @@ __device__ __forceinline__ float full_dist(const float (&k)[D], const uint8_t* r
     return __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
 }
 
+// acc + x*x for the bf16 x in the low / high half of w, rounded once (sm_100
+// mixed-precision fma; x*x is exact in fp32, so this equals fmaf on the
+// widened value)
+__device__ __forceinline__ float sqacc_lo(uint32_t w, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, l, l, %2;\n\t}" : "=f"(r) : "r"(w), "f"(acc));
+    return r;
+}
+__device__ __forceinline__ float sqacc_hi(uint32_t w, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, h, h, %2;\n\t}" : "=f"(r) : "r"(w), "f"(acc));
+    return r;
+}
+
+// Three-input fp32 minimum (sm_100).
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // NWG independent 128-thread pipelines (warpgroups) per CTA, one thread per
-// key; each has its own K/V staging, TMEM buffer and mbarriers, and they share
-// the per-head parent image, children image, norms and counts. SEP: separate K
-// and V stages per warpgroup (V of a tile lands while its K is in use);
-// otherwise one stage that holds the tile's K until the key rows are in
-// registers and then its V (d = 128, where two stages do not fit).
-template <int D, int C, int NWG, bool SEP>
+// key. Each warpgroup has its own K stage, TMEM accumulator and mbarriers
+// and meets its own threads once per tile; the warpgroups share the per-head
+// parent image, children image, norms and counts, and meet CTA-wide only
+// where the (batch, head) changes.
+template <int D, int C, int NWG>
 __global__ void __launch_bounds__(128 * NWG, 1)
-precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmCB, const TcPreParams p) {
+precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmCB,
+                     const TcPreParams p) {
     constexpr int KH = D / 64;
     constexpr uint32_t IMG = KH * kRegion;
     constexpr int KSTEPS = D / 16;
     constexpr int NT = 128 * NWG;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = align1024p(smem_raw);
-    constexpr int NSTAGE = SEP ? 2 * NWG : NWG;
     uint8_t* sK0 = base;                           // K stage of warpgroup w: sK0 + w*IMG
-    uint8_t* sV0 = SEP ? base + NWG * IMG : base;  // V stage of warpgroup w: sV0 + w*IMG
-    uint8_t* sB1 = base + NSTAGE * IMG;            // parent codewords (K-major, TMA), M0p rows
+    uint8_t* sB1 = base + NWG * IMG;               // parent codewords (K-major, TMA), M0p rows
     const uint32_t b1_region = (uint32_t)p.M0p * 128u;   // bytes between its 64-column blocks
-    uint8_t* sCh = sB1 + KH * b1_region;     // children image [M0*C rows x D] bf16
+    uint8_t* sCh = sB1 + KH * b1_region;           // children image [M0*C rows x D] bf16
     const size_t ch_bytes = (size_t)p.M0 * C * D * 2;
     float* sCn = reinterpret_cast<float*>(sCh + ((ch_bytes + 15) & ~size_t(15)));   // [128]
-    int* sPar = reinterpret_cast<int*>(sCn + 128);           // [NWG][128]
-    int* sLeaf = sPar + 128 * NWG;                           // [NWG][128]
-    float* sRed = reinterpret_cast<float*>(sLeaf + 128 * NWG);   // [8]
-    int* sCnt = reinterpret_cast<int*>(sRed + 8);            // [Mtot]
+    float* sRed = sCn + 128;                       // [4]
+    int* sCnt = reinterpret_cast<int*>(sRed + 4);  // [Mtot]
     uint64_t* bars = reinterpret_cast<uint64_t*>(
         (reinterpret_cast<uintptr_t>(sCnt + p.Mtot) + 7) & ~uintptr_t(7));
-    // bars: per warpgroup w: 3w+0 = K stage, 3w+1 = V stage, 3w+2 = MMA; 3*NWG = head
-    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 3 * NWG + 1);
+    // bars: per warpgroup w: 2w = K stage, 2w+1 = MMA; 2*NWG = head
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 2 * NWG + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wg = tid >> 7, lt = tid & 127;        // warpgroup, key row within the tile
     const int wgbar = 1 + wg;
-    uint64_t* barK = &bars[3 * wg];
-    uint64_t* barV = &bars[3 * wg + 1];
-    uint64_t* barM = &bars[3 * wg + 2];
-    uint64_t* barH = &bars[3 * NWG];
+    uint64_t* barK = &bars[2 * wg];
+    uint64_t* barM = &bars[2 * wg + 1];
+    uint64_t* barH = &bars[2 * NWG];
     uint8_t* sK = sK0 + wg * IMG;
-    uint8_t* sV = sV0 + wg * IMG;
-    int* myPar = sPar + 128 * wg;
-    int* myLeaf = sLeaf + 128 * wg;
     const int g0 = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
     const int g1 = (int)(((long long)(blockIdx.x + 1) * p.total_tiles) / gridDim.x);
 
     if (warp == 0) {
-        tmem_alloc(sTmem, 128 * NWG < 32 ? 32 : 128 * NWG);
+        tmem_alloc(sTmem, 128 * NWG);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 3 * NWG + 1; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2 * NWG + 1; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmCB);
     }
     for (int i = tid; i < p.Mtot; i += NT) sCnt[i] = 0;
@@ -221,7 +260,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     // ||k||^2 + max ||C_p||^2)
     const float c_exp = 2.f * (5.f * D + 8.f) * 5.9604644775390625e-08f;
 
-    uint32_t kph = 0, vph = 0, mph = 0, hph = 0;
+    uint32_t kph = 0, mph = 0, hph = 0;
     bool failed = false;
     int cur_bh = -1;
     float cnmax = 0.f;
@@ -232,12 +271,6 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         mbar_arrive_expect_tx(barK, IMG);
 #pragma unroll
         for (int kh = 0; kh < KH; ++kh) tma_load_3d(sK + kh * kRegion, &tmK, barK, kh * 64, t * kTile, bh);
-    };
-    auto issue_v = [&](int g) {
-        const int bh = g / p.ntiles, t = g % p.ntiles;
-        mbar_arrive_expect_tx(barV, IMG);
-#pragma unroll
-        for (int kh = 0; kh < KH; ++kh) tma_load_3d(sV + kh * kRegion, &tmV, barV, kh * 64, t * kTile, bh);
     };
     auto flush_counts = [&](int bh) {
         for (int i = tid; i < p.Mtot; i += NT) {
@@ -253,7 +286,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         // segment [gs, ge): the tiles of one (b,h) in this CTA's range
         const int bh = gs / p.ntiles, h = bh % p.H;
         const int ge = min(g1, (bh + 1) * p.ntiles);
-        __syncthreads();   // both warpgroups are done with the previous segment
+        __syncthreads();   // every warpgroup is done with the previous segment
         if (cur_bh >= 0) flush_counts(cur_bh);
         bool ok = true;
         if (cur_bh < 0 || h != cur_bh % p.H) {
@@ -268,35 +301,38 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                 cp_async_16(sCh + ch_off<D>(i, i / C, j), chg + (size_t)i * D + j * 8);
             }
             cp_async_commit();
-            float cn = 0.f;
-            if (tid < p.M0) {
-                const uint16_t* cp = p.codebook + ((size_t)h * p.Mtot + tid) * D;
-#pragma unroll 8
-                for (int j = 0; j < D; ++j) {
-                    const float c = __uint_as_float((uint32_t)__ldg(cp + j) << 16);
-                    cn = __fmaf_rn(c, c, cn);
-                }
-            }
-            // ||C_p||^2 is +inf for padding parents (p >= M0): they never win
-            if (tid < 128) sCn[tid] = tid < p.M0 ? cn : INFINITY;
-            float mx = cn;
-#pragma unroll
-            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) sRed[warp] = mx;
-            cp_async_wait_all();
-            fence_proxy_async_smem();
             ok = mbar_wait(barH, hph);
             hph ^= 1;
+            // ||C_p||^2 from the parent image, terms in index order; +inf for
+            // padding parents (p >= M0): they never win
+            if (tid < 128) {
+                float cn = 0.f;
+                if (tid < p.M0 && ok) {
+#pragma unroll
+                    for (int j = 0; j < D / 8; ++j) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(sB1 + swz_off(tid, j, b1_region));
+                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            cn = __fmaf_rn(bf_lo(ww[e]), bf_lo(ww[e]), cn);
+                            cn = __fmaf_rn(bf_hi(ww[e]), bf_hi(ww[e]), cn);
+                        }
+                    }
+                }
+                sCn[tid] = tid < p.M0 ? cn : INFINITY;
+                float mx = cn;
+#pragma unroll
+                for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                if (lane == 0) sRed[warp] = mx;
+            }
+            cp_async_wait_all();
         }
         if (__syncthreads_or(!ok)) { failed = true; break; }
         cnmax = fmaxf(fmaxf(sRed[0], sRed[1]), fmaxf(sRed[2], sRed[3]));
         cur_bh = bh;
 
         // this warpgroup's tiles of the segment
-        if (lt == 0 && gs + wg < ge) {
-            issue_k(gs + wg);
-            if (SEP) issue_v(gs + wg);
-        }
+        if (lt == 0 && gs + wg < ge) issue_k(gs + wg);
         for (int g = gs + wg; g < ge; g += NWG) {
             const int t = g % p.ntiles;
             const int rows = min(kTile, p.N - t * kTile);
@@ -318,83 +354,73 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             // (if thread lt 0 could not issue the MMA, every thread's wait below times out)
             ok = mbar_wait(barM, mph) && ok;
             mph ^= 1;
-            if (wg_sync_or(wgbar, !ok)) { failed = true; break; }
             tc_fence_after();
 
-            // key row -> fp32 registers; ||k||^2
-            float k[D];
+            // ---- a1, pass 1: the smallest v_p = ||C_p||^2 - 2 S_p
+            float m = INFINITY;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (16 * c < p.M0p) {
+                    float v16[16];
+                    tmem_ld16f(trow + 16 * c, v16);
+                    tmem_wait_ld();
+                    tmem_touch16f(v16);
+#pragma unroll
+                    for (int q = 0; q < 16; q += 4) {
+                        const float4 cn4 = *reinterpret_cast<const float4*>(sCn + 16 * c + q);
+                        m = fmin3(m, fmaf(-2.f, v16[q], cn4.x), fmaf(-2.f, v16[q + 1], cn4.y));
+                        m = fmin3(m, fmaf(-2.f, v16[q + 2], cn4.z), fmaf(-2.f, v16[q + 3], cn4.w));
+                    }
+                }
+            }
+
+            // ||k||^2 straight from the bf16 key row (the row itself is
+            // loaded again once the parent is known, to keep registers free)
             float kn;
             {
                 float kn0 = 0.f, kn1 = 0.f;
 #pragma unroll
                 for (int j = 0; j < D / 8; ++j) {
                     const uint4 w = *reinterpret_cast<const uint4*>(sK + swz_off(lt, j));
-                    k[8 * j + 0] = bf_lo(w.x); k[8 * j + 1] = bf_hi(w.x);
-                    k[8 * j + 2] = bf_lo(w.y); k[8 * j + 3] = bf_hi(w.y);
-                    k[8 * j + 4] = bf_lo(w.z); k[8 * j + 5] = bf_hi(w.z);
-                    k[8 * j + 6] = bf_lo(w.w); k[8 * j + 7] = bf_hi(w.w);
-#pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        kn0 = __fmaf_rn(k[8 * j + e], k[8 * j + e], kn0);
-                        kn1 = __fmaf_rn(k[8 * j + e + 1], k[8 * j + e + 1], kn1);
-                    }
+                    kn0 = sqacc_lo(w.x, kn0); kn1 = sqacc_hi(w.x, kn1);
+                    kn0 = sqacc_lo(w.y, kn0); kn1 = sqacc_hi(w.y, kn1);
+                    kn0 = sqacc_lo(w.z, kn0); kn1 = sqacc_hi(w.z, kn1);
+                    kn0 = sqacc_lo(w.w, kn0); kn1 = sqacc_hi(w.w, kn1);
                 }
                 kn = __fadd_rn(kn0, kn1);
             }
-            if (!SEP) {   // the stage now takes this tile's V
-                wg_sync(wgbar);
-                if (lt == 0) issue_v(g);
-            }
 
-            // ---- a1: nearest parent; four trackers over interleaved columns
-            float best, second;
-            int bp;
-            {
-                float bu[4], su[4];
-                int pu[4];
+            // ---- a1, pass 2: the parents within the error band of the
+            // smallest (count in the low byte, their index sum above it); a
+            // single one is certainly the nearest
+            const float E = c_exp * (kn + cnmax);
+            const float thr = __fadd_ru(m, 2.f * E);
+            int acc = 0;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) { bu[u] = INFINITY; su[u] = INFINITY; pu[u] = 0x7fffffff; }
+            for (int c = 0; c < 8; ++c) {
+                if (16 * c < p.M0p) {
+                    float v16[16];
+                    tmem_ld16f(trow + 16 * c, v16);
+                    tmem_wait_ld();
+                    tmem_touch16f(v16);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (16 * c < p.M0p) {
-                        float v16[16];
-                        tmem_ld16f(trow + 16 * c, v16);
-                        tmem_wait_ld();
-                        tmem_touch16f(v16);
+                    for (int q = 0; q < 16; q += 4) {
+                        const float4 cn4 = *reinterpret_cast<const float4*>(sCn + 16 * c + q);
+                        const float cnq[4] = {cn4.x, cn4.y, cn4.z, cn4.w};
 #pragma unroll
-                        for (int q = 0; q < 16; q += 4) {
-                            const float4 cn4 = *reinterpret_cast<const float4*>(sCn + 16 * c + q);
-                            const float cnq[4] = {cn4.x, cn4.y, cn4.z, cn4.w};
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const float v = fmaf(-2.f, v16[q + u], cnq[u]);
-                                if (v < bu[u]) { su[u] = bu[u]; bu[u] = v; pu[u] = 16 * c + q + u; }
-                                else su[u] = fminf(su[u], v);
-                            }
-                        }
+                        for (int u = 0; u < 4; ++u)
+                            if (fmaf(-2.f, v16[q + u], cnq[u]) <= thr) acc += ((16 * c + q + u) << 8) + 1;
                     }
                 }
-#pragma unroll
-                for (int u = 1; u < 4; ++u) {
-                    const bool take = (bu[u] < bu[0]) || (bu[u] == bu[0] && pu[u] < pu[0]);
-                    const float lo = take ? bu[u] : bu[0], hi = take ? bu[0] : bu[u];
-                    su[0] = fminf(hi, fminf(su[0], su[u]));
-                    bu[0] = lo;
-                    pu[0] = take ? pu[u] : pu[0];
-                }
-                best = bu[0];
-                second = su[0];
-                bp = pu[0] < p.M0 ? pu[0] : 0;
             }
-            const uint16_t* cbh = p.codebook + (size_t)h * p.Mtot * D;
-            const uint16_t* krow = p.K + ((size_t)bh * p.N + (size_t)t * kTile + lt) * D;
-            const float E = c_exp * (kn + cnmax);
-            const bool redecide = valid && p.M0 > 1 && !(second - best > 2.f * E);
+            int bp = (acc & 255) == 1 ? (acc >> 8) : 0;
+            const bool redecide = valid && (acc & 255) != 1;
             if (__any_sync(0xffffffffu, redecide)) {
-                // re-decide among the parents within the band, in fp64 (TMEM
-                // reloads are warp-wide, the fp64 work only where needed)
+                // exact fp64 distances of the parents within the band, in
+                // index order (TMEM reloads are warp-wide, the fp64 work only
+                // where needed)
                 double eb = INFINITY;
-                int ep = bp;
+                int ep = 0;
                 for (int c = 0; c < p.M0p; c += 16) {
                     float v16[16];
                     tmem_ld16f(trow + c, v16);
@@ -404,9 +430,10 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                         for (int q = 0; q < 16; ++q) {
                             const int pp = c + q;
                             if (pp >= p.M0) break;
-                            const float v = fmaf(-2.f, v16[q], sCn[pp]);
-                            if (v - best > 2.f * E) continue;
-                            const double e = exact_dist_glob<D>(krow, cbh + (size_t)pp * D);
+                            if (!(fmaf(-2.f, v16[q], sCn[pp]) <= thr)) continue;
+                            const double e = exact_dist_smem<D>(
+                                sK, [&](int j) { return swz_off(lt, j); }, sB1,
+                                [&](int j) { return swz_off(pp, j, b1_region); });
                             if (e < eb) { eb = e; ep = pp; }
                         }
                     }
@@ -416,90 +443,112 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                     ++n_pre;
                 }
             }
+            // key row -> fp32 registers
+            float k[D];
+#pragma unroll
+            for (int j = 0; j < D / 8; ++j) {
+                const uint4 w = *reinterpret_cast<const uint4*>(sK + swz_off(lt, j));
+                k[8 * j + 0] = bf_lo(w.x); k[8 * j + 1] = bf_hi(w.x);
+                k[8 * j + 2] = bf_lo(w.y); k[8 * j + 3] = bf_hi(w.y);
+                k[8 * j + 4] = bf_lo(w.z); k[8 * j + 5] = bf_hi(w.z);
+                k[8 * j + 6] = bf_lo(w.w); k[8 * j + 7] = bf_hi(w.w);
+            }
+            tc_fence_before();   // this tile's TMEM reads before the next MMA into the buffer
+            if (wg_sync_or(wgbar, !ok)) { failed = true; break; }   // also: the K stage is free
+            if (lt == 0 && g + NWG < ge) issue_k(g + NWG);
 
-            // ---- a2: the kept parent and its children, direct form
+            // ---- a2: the kept parent and its children, direct form. A child
+            // wins only when strictly closer (parent first, lowest child index
+            // among equals); the runner-up decides whether the bound separates
+            // the winner from every other candidate (the test is monotone in
+            // the runner-up's distance).
             int leaf = bp;
             {
                 const float dpar = full_dist<D>(k, sB1, [&](int j) { return swz_off(bp, j, b1_region); });
-                float dch[C];
-                float lo = dpar;
+                float lo = dpar, sec = INFINITY;
                 int lo_i = -1;
 #pragma unroll
                 for (int c = 0; c < C; ++c) {
                     const int i = bp * C + c;
-                    dch[c] = full_dist<D>(k, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
-                    if (dch[c] < lo) { lo = dch[c]; lo_i = c; }
+                    const float dc = full_dist<D>(k, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
+                    if (dc < lo) { sec = lo; lo = dc; lo_i = c; }
+                    else sec = fminf(sec, dc);
                 }
-                bool sure = (lo_i < 0) || separated(lo, dpar, eps_dir);
-#pragma unroll
-                for (int c = 0; c < C; ++c)
-                    if (c != lo_i && !separated(lo, dch[c], eps_dir)) sure = false;
-                if (sure || !valid) {
+                if (separated(lo, sec, eps_dir) || !valid) {
                     leaf = lo_i < 0 ? bp : p.M0 + bp * C + lo_i;
                 } else {
-                    double eb = exact_dist_glob<D>(krow, cbh + (size_t)bp * D);
-                    int win = bp;
-#pragma unroll
+                    // fp64 among the parent and the children within the band
+                    // (the key row comes back from global memory: its stage
+                    // may already hold the next tile)
+                    uint32_t band = 0;
                     for (int c = 0; c < C; ++c) {
-                        if (separated(lo, dch[c], eps_dir)) continue;
-                        const double e = exact_dist_glob<D>(krow, cbh + (size_t)(p.M0 + bp * C + c) * D);
-                        if (e < eb) { eb = e; win = p.M0 + bp * C + c; }
+                        const int i = bp * C + c;
+                        const float dc = full_dist<D>(k, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
+                        if (!separated(lo, dc, eps_dir)) band |= 1u << c;
+                    }
+                    const uint16_t* krow = p.K + ((size_t)bh * p.N + (size_t)t * kTile + lt) * D;
+                    double eb = exact_dist_gk<D>(krow, sB1, [&](int j) { return swz_off(bp, j, b1_region); });
+                    int win = bp;
+                    for (; band; band &= band - 1) {
+                        const int i = bp * C + __ffs(band) - 1;
+                        const double e = exact_dist_gk<D>(krow, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
+                        if (e < eb) { eb = e; win = p.M0 + i; }
                     }
                     leaf = win;
                     ++n_chd;
                 }
             }
 
-            // ---- a3: outputs
-            if (valid) {
-                p.assign[(size_t)bh * p.N + t * kTile + lt] = leaf;
-                atomicAdd(&sCnt[bp], 1);
-                if (leaf != bp) atomicAdd(&sCnt[leaf], 1);
+            // ---- a3: outputs. Counts and value sums go to the leaf only (the
+            // parent itself or the child); the parents' totals are completed
+            // by adding their children's when all tiles are done.
+            const int kl = valid ? leaf : -1;
+            if (valid) p.assign[(size_t)bh * p.N + t * kTile + lt] = leaf;
+            {
+                const unsigned same = __match_any_sync(0xffffffffu, kl);
+                if (valid && lane == __ffs(same) - 1) atomicAdd(&sCnt[leaf], __popc(same));
             }
-            myPar[lt] = valid ? bp : -1;
-            myLeaf[lt] = leaf;
-            const bool ok_v = mbar_wait(barV, vph);
-            vph ^= 1;
-            tc_fence_before();   // TMEM reads of this tile before the next MMA into the buffer
-            if (wg_sync_or(wgbar, !ok_v)) { failed = true; break; }   // also: K stage free (SEP)
-            if (SEP && lt == 0 && g + NWG < ge) issue_k(g + NWG);
-
-            // value sums: warp (w%4) adds the V rows of keys 32(w%4)..+31, two
-            // keys per step (one per half-warp), 16-byte vector reductions
+            // value sums: two keys of this warp per step (one per half-warp),
+            // the V row read straight from global memory (coalesced), 16-byte
+            // fp32 vector reductions
             {
                 const int hl = lane & 15, sub = lane >> 4;
-                constexpr int DPL = D / 16;                       // dimensions per lane
-                const int j = (hl * DPL) >> 3;                    // 16-byte chunk of those dimensions
-                const uint32_t inchunk = ((hl * DPL) & 7) * 2;    // byte offset inside the chunk
+                constexpr int DPL = D / 16;   // dimensions per lane
+                const size_t row0 = (size_t)bh * p.N + (size_t)t * kTile + 32 * (warp & 3);
+                const uint16_t* vsrc = p.V + row0 * D + hl * DPL;
                 float* vs_lane = p.vsum + (size_t)bh * p.Mtot * D + hl * DPL;
-#pragma unroll 4
-                for (int q = 0; q < 16; ++q) {
-                    const int rr = 32 * (warp & 3) + 2 * q + sub;
-                    const int par = myPar[rr];
-                    const int lf = myLeaf[rr];
-                    if (par >= 0) {
-                        const uint8_t* src = sV + swz_off(rr, j) + inchunk;
-                        if (D == 64) {
-                            const uint2 w = *reinterpret_cast<const uint2*>(src);
-                            const float a = bf_lo(w.x), b = bf_hi(w.x), c = bf_lo(w.y), d = bf_hi(w.y);
-                            red_v4(vs_lane + (size_t)par * D, a, b, c, d);
-                            if (lf != par) red_v4(vs_lane + (size_t)lf * D, a, b, c, d);
-                        } else {
-                            const uint4 w = *reinterpret_cast<const uint4*>(src);
-                            red_v4(vs_lane + (size_t)par * D, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-                            red_v4(vs_lane + (size_t)par * D + 4, bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
-                            if (lf != par) {
-                                red_v4(vs_lane + (size_t)lf * D, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-                                red_v4(vs_lane + (size_t)lf * D + 4, bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
-                            }
+                if (D == 64) {
+                    uint2 w[16];
+                    int lf[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        lf[q] = __shfl_sync(0xffffffffu, kl, 2 * q + sub);
+                        w[q] = make_uint2(0u, 0u);
+                        if (lf[q] >= 0) w[q] = __ldg(reinterpret_cast<const uint2*>(vsrc + (size_t)(2 * q + sub) * D));
+                    }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (lf[q] >= 0)
+                            red_v4(vs_lane + (size_t)lf[q] * D, bf_lo(w[q].x), bf_hi(w[q].x), bf_lo(w[q].y),
+                                   bf_hi(w[q].y));
+                } else {
+                    uint4 w[16];
+                    int lf[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        lf[q] = __shfl_sync(0xffffffffu, kl, 2 * q + sub);
+                        w[q] = make_uint4(0u, 0u, 0u, 0u);
+                        if (lf[q] >= 0) w[q] = __ldg(reinterpret_cast<const uint4*>(vsrc + (size_t)(2 * q + sub) * D));
+                    }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        if (lf[q] >= 0) {
+                            float* dst = vs_lane + (size_t)lf[q] * D;
+                            red_v4(dst, bf_lo(w[q].x), bf_hi(w[q].x), bf_lo(w[q].y), bf_hi(w[q].y));
+                            red_v4(dst + 4, bf_lo(w[q].z), bf_hi(w[q].z), bf_lo(w[q].w), bf_hi(w[q].w));
                         }
                     }
                 }
-            }
-            wg_sync(wgbar);   // V stage free, myPar/myLeaf reusable
-            if (lt == 0 && g + NWG < ge) {
-                if (SEP) issue_v(g + NWG);
-                else issue_k(g + NWG);
             }
         }
         if (__syncthreads_or(failed)) { failed = true; break; }
@@ -518,17 +567,45 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128 * NWG < 32 ? 32 : 128 * NWG);
+        tmem_dealloc(tmem, 128 * NWG);
     }
 }
 
+// Completes the parents' totals: counts[p] and vsum[p] (which so far hold the
+// keys that stayed at the parent) plus those of the parent's C children. One
+// warp per (b, h, parent).
+template <int D, int C>
+__global__ void __launch_bounds__(256) precompute_parent_totals_kernel(int BHM0, int M0, int Mtot, int32_t* counts,
+                                                                       float* vsum) {
+    const int w = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (w >= BHM0) return;
+    const int bh = w / M0, pp = w % M0;
+    const size_t prow = (size_t)bh * Mtot + pp;
+    const size_t crow = (size_t)bh * Mtot + M0 + (size_t)pp * C;
+    constexpr int DL = D / 32;   // dimensions per lane (2 or 4)
+    float acc[DL];
+#pragma unroll
+    for (int e = 0; e < DL; ++e) acc[e] = vsum[prow * D + lane * DL + e];
+    int cnt = 0;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+#pragma unroll
+        for (int e = 0; e < DL; ++e) acc[e] += vsum[(crow + c) * D + lane * DL + e];
+        cnt += counts[crow + c];
+    }
+#pragma unroll
+    for (int e = 0; e < DL; ++e) vsum[prow * D + lane * DL + e] = acc[e];
+    if (lane == 0) counts[prow] += cnt;
+}
+
+int pre_nwg(int D) { return D == 64 ? 4 : 2; }
+
 size_t pre_smem_bytes(int D, int M0, int C, int Mtot) {
-    const int nwg = 2;
-    const int nstage = D == 64 ? 2 * nwg : nwg;
+    const int nwg = pre_nwg(D);
     const size_t M0p = (size_t)((M0 + 15) & ~15);
-    return 1024 + nstage * (size_t)(D / 64) * kRegion + (size_t)(D / 64) * M0p * 128 +
-           (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) + 128 * 4 /*sCn*/ + 2 * nwg * 128 * 4 /*sPar, sLeaf*/ +
-           8 * 4 + (size_t)Mtot * 4 + 8 + (3 * nwg + 1) * 8 + 16;
+    return 1024 + nwg * (size_t)(D / 64) * kRegion + (size_t)(D / 64) * M0p * 128 +
+           (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) + 128 * 4 /*sCn*/ + 4 * 4 /*sRed*/ + (size_t)Mtot * 4 +
+           8 + (2 * nwg + 1) * 8 + 16;
 }
 
 template <int D, int C>
@@ -537,8 +614,8 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     const int BH = s.B * s.H;
     const int Mtot = s.M0 * (1 + s.C);
     const int M0p = (s.M0 + 15) & ~15;
-    CUtensorMap tk, tv, tcb;
-    if (!make_tma_bf16_3d(&tk, K, D, s.N, BH, kTile) || !make_tma_bf16_3d(&tv, V, D, s.N, BH, kTile) ||
+    CUtensorMap tk, tcb;
+    if (!make_tma_bf16_3d(&tk, K, D, s.N, BH, kTile) ||
         !make_tma_bf16_3d(&tcb, cb, D, Mtot, s.H, M0p))
         return cudaErrorInvalidValue;
     TcPreParams prm;
@@ -551,21 +628,27 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     prm.ntiles = (s.N + kTile - 1) / kTile;
     prm.total_tiles = prm.ntiles * BH;
     prm.K = static_cast<const uint16_t*>(K);
+    prm.V = static_cast<const uint16_t*>(V);
     prm.codebook = static_cast<const uint16_t*>(cb);
     prm.assign = assign;
     prm.counts = counts;
     prm.vsum = vsum;
     prm.status = status;
     const size_t smem = pre_smem_bytes(D, s.M0, C, Mtot);
-    constexpr int NWG = 2;
-    auto kern = precompute_tc_kernel<D, C, NWG, D == 64>;
+    constexpr int NWG = D == 64 ? 4 : 2;
+    auto kern = precompute_tc_kernel<D, C, NWG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = std::min(prm.total_tiles, sms);
-    kern<<<grid, 128 * NWG, smem, st>>>(tk, tv, tcb, prm);
+    kern<<<grid, 128 * NWG, smem, st>>>(tk, tcb, prm);
+    count_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int warps = BH * s.M0;
+    precompute_parent_totals_kernel<D, C><<<(warps + 7) / 8, 256, 0, st>>>(warps, s.M0, Mtot, counts, vsum);
     count_launch();
     return cudaGetLastError();
 }
