@@ -69,6 +69,39 @@ __device__ __forceinline__ uint32_t swz(int r, int j) {
     return (uint32_t)(j >> 3) * kRegion + (uint32_t)r * 128u + (uint32_t)(((j & 7) ^ (r & 7)) << 4);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes
+// of data, each element rounded as its scalar counterpart.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// Three-input fp32 maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Sum of each of 64 columns over the 32 lanes of a warp (a butterfly that
 // halves the number of values each step): on return lane L holds the sums of
 // columns 2L and 2L+1 in v[0], v[1].
@@ -139,7 +172,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     float* sLb = reinterpret_cast<float*>(base + 6 * IMG);   // [128] log2 n_p (-inf if empty)
     float* sInvN = sLb + 128;                                // [128] 1 / n_p
     float* sNc = sInvN + 128;                                // [128] child counts of the chunk
-    float* sPart = sNc + 128;                                // [4][128] importance partials
+    float* sLc = sNc + 128;                                  // [128] their log2 (-inf if empty)
+    float* sPart = sLc + 128;                                // [4][128] importance partials
     float* sX = sPart + 512;                                 // [2][128] row exchange (max, Zbar, den)
     int* sRank = reinterpret_cast<int*>(sX + 256);           // [2][128] partial ranks
     unsigned long long* sKey = reinterpret_cast<unsigned long long*>(sRank + 256);   // [128]
@@ -253,43 +287,53 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tmem_wait_ld();
 #pragma unroll
         for (int b = 0; b < 4; ++b) tmem_touch16f(x + 16 * b);
-        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const float2 sl2v = make_float2(p.sl2, p.sl2);
+        float mp0 = -INFINITY, mp1 = -INFINITY;
 #pragma unroll
         for (int k = 0; k < 64; k += 4) {
             const float4 lb = *reinterpret_cast<const float4*>(sLb + 32 * (k >> 4) + 16 * hf + (k & 15));
-            x[k + 0] = fmaf(x[k + 0], p.sl2, lb.x);
-            x[k + 1] = fmaf(x[k + 1], p.sl2, lb.y);
-            x[k + 2] = fmaf(x[k + 2], p.sl2, lb.z);
-            x[k + 3] = fmaf(x[k + 3], p.sl2, lb.w);
-            mp[(k >> 2) & 3] = fmaxf(mp[(k >> 2) & 3], fmaxf(fmaxf(x[k], x[k + 1]), fmaxf(x[k + 2], x[k + 3])));
+            const float2 a = ffma2(make_float2(x[k], x[k + 1]), sl2v, make_float2(lb.x, lb.y));
+            const float2 b = ffma2(make_float2(x[k + 2], x[k + 3]), sl2v, make_float2(lb.z, lb.w));
+            x[k] = a.x; x[k + 1] = a.y; x[k + 2] = b.x; x[k + 3] = b.y;
+            mp0 = fmax3(mp0, a.x, a.y);
+            mp1 = fmax3(mp1, b.x, b.y);
         }
-        sX[hf * 128 + r] = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        sX[hf * 128 + r] = fmaxf(mp0, mp1);
         pair_sync(quarter);
         const float m = fmaxf(sX[r], sX[128 + r]);
         pair_sync(quarter);
-        float zp[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 negm = make_float2(-m, -m);
+        float2 zp0 = make_float2(0.f, 0.f), zp1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             uint32_t w[8], e[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float ev = ex2(x[16 * c + k] - m);   // = A_p n_p (0 for empty parents)
-                x[16 * c + k] = ev;
-                zp[k & 3] += ev;
-                e[k] = __float_as_uint(ev);
+            for (int k = 0; k < 16; k += 2) {
+                const float2 tt = fadd2(make_float2(x[16 * c + k], x[16 * c + k + 1]), negm);
+                const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));   // = A_p n_p (0 for empty parents)
+                x[16 * c + k] = ev.x;
+                x[16 * c + k + 1] = ev.y;
+                if ((k >> 1) & 1) zp1 = fadd2(zp1, ev);
+                else zp0 = fadd2(zp0, ev);
+                e[k] = __float_as_uint(ev.x);
+                e[k + 1] = __float_as_uint(ev.y);
+                w[k >> 1] = pack_bf16x2(ev.x, ev.y);
             }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) w[k] = pack_bf16x2(x[16 * c + 2 * k], x[16 * c + 2 * k + 1]);
             tmem_st8(trow + p.colW + 16 * c + 8 * hf, w);     // bf16 weights: A operand of MMA3
             tmem_st16(trow + 32 * c + 16 * hf, e);            // fp32 e'_p kept for the child pass
         }
-        sX[hf * 128 + r] = (zp[0] + zp[1]) + (zp[2] + zp[3]);
+        sX[hf * 128 + r] = (zp0.x + zp0.y) + (zp1.x + zp1.y);
         pair_sync(quarter);
         const float z = sX[r] + sX[128 + r];
         // importance terms e'_p / Zbar_i (zero for rows past the end)
         const float rz = valid ? 1.f / z : 0.f;
+        const float2 rz2 = make_float2(rz, rz);
 #pragma unroll
-        for (int k = 0; k < 64; ++k) x[k] *= rz;
+        for (int k = 0; k < 64; k += 2) {
+            const float2 v = fmul2(make_float2(x[k], x[k + 1]), rz2);
+            x[k] = v.x;
+            x[k + 1] = v.y;
+        }
         butterfly_colsum64(x, lane);
         // lane L now holds the row-block sums of this half's x[2L], x[2L+1], i.e.
         // of parent columns 32(L/8) + 16hf + 2(L%8) and the next one
@@ -337,13 +381,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
 
         // ---- children, in chunks of <= 128 slots (this half: slots 64hf..64hf+63)
-        float denp[4] = {0.f, 0.f, 0.f, 0.f};   // child corrections of the denominator
+        float2 den0 = make_float2(0.f, 0.f), den1 = make_float2(0.f, 0.f);   // child corrections of the denominator
         const int PC = p.P * C;
         const int nchunks = (PC + kTile - 1) / kTile;
         for (int k = 0; k < nchunks; ++k) {
             const int s0 = k * kTile;
             const int ns = min(kTile, PC - s0);
-            const int N2 = (ns + 15) & ~15;
+            const int N2 = (ns + 31) & ~31;   // whole 32-slot blocks: every column read is written
             for (int idx = tid; idx < N2 * (D / 8); idx += 256) {
                 const int slot = idx / (D / 8), j = idx % (D / 8);
                 const uint32_t off = swz(slot, j);
@@ -365,10 +409,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     nc = (float)__ldg(p.counts + (size_t)bh * p.Mtot + p.M0 + sSel[sg / C] * C + (sg % C));
                 }
                 sNc[tid] = nc;
+                sLc[tid] = nc > 0.f ? __log2f(nc) : -INFINITY;
             }
-            // A_p = e'_p / n_p of the parents behind this half's two slot blocks,
-            // read before MMA2 may reuse the columns
-            float ap[2][PPB];
+            // -A_p = -e'_p / n_p of the parents behind this half's two slot
+            // blocks, read before MMA2 may reuse the columns
+            float nap[2][PPB];
             {
                 uint32_t rr[2][PPB];
 #pragma unroll
@@ -382,8 +427,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                     for (int q = 0; q < PPB; ++q) {
                         tmem_touch1(rr[c][q]);
-                        ap[c][q] = __uint_as_float(rr[c][q]) *
-                                   sInvN[sSel[min((s0 + 64 * c + 32 * hf) / C + q, p.P - 1)]];
+                        nap[c][q] = -__uint_as_float(rr[c][q]) *
+                                    sInvN[sSel[min((s0 + 64 * c + 32 * hf) / C + q, p.P - 1)]];
                     }
             }
             cp_async_wait_all();
@@ -403,7 +448,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (__syncthreads_or(!ok)) { failed = true; break; }
             tc_fence_after();
 
-            // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m) for this half's slots
+            // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m) for this half's
+            // slots, as 2^(sl2*S - m + log2 n_c) - A_p n_c (empty and padding
+            // slots: 0 - A_p * 0)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 const int sb = 64 * c + 32 * hf;                   // first slot of this block
@@ -412,20 +459,22 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tmem_ld32f(trow + p.colSc + sb, sc);
                 uint32_t w[16];
 #pragma unroll
-                for (int kk = 0; kk < 32; kk += 2) {
-                    float dd[2];
+                for (int kk = 0; kk < 32; kk += 4) {
+                    const float4 lc = *reinterpret_cast<const float4*>(sLc + sb + kk);
+                    const float4 nc = *reinterpret_cast<const float4*>(sNc + sb + kk);
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int j = kk + e;                      // slot within the block
-                        const float nc = sNc[sb + j];
-                        const float xc = fminf(fmaf(sc[kk + e], p.sl2, -m), 126.f);
-                        xmax = fmaxf(xmax, nc > 0.f ? xc : -INFINITY);
-                        // slots past the chunk hold stale TMEM columns: their weight is 0
-                        const float wc = nc > 0.f ? (ex2(xc) - ap[c][j / C]) * nc : 0.f;
-                        denp[(kk >> 1) & 3] += wc;
-                        dd[e] = wc;
+                        const int j = kk + 2 * e;                  // slot within the block
+                        float2 tt = ffma2(make_float2(sc[j], sc[j + 1]), sl2v, negm);
+                        tt = fadd2(tt, e ? make_float2(lc.z, lc.w) : make_float2(lc.x, lc.y));
+                        xmax = fmax3(xmax, tt.x, tt.y);
+                        const float2 ev = make_float2(ex2(fminf(tt.x, 126.f)), ex2(fminf(tt.y, 126.f)));
+                        const float2 wc = ffma2(make_float2(nap[c][j / C], nap[c][(j + 1) / C]),
+                                                e ? make_float2(nc.z, nc.w) : make_float2(nc.x, nc.y), ev);
+                        if (e) den1 = fadd2(den1, wc);
+                        else den0 = fadd2(den0, wc);
+                        w[j >> 1] = pack_bf16x2(wc.x, wc.y);
                     }
-                    w[kk / 2] = pack_bf16x2(dd[0], dd[1]);
                 }
                 tmem_st16(trow + p.colWc + (sb >> 1), w);
             }
@@ -453,20 +502,23 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
 
         // ---- epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
-        sX[hf * 128 + r] = (denp[0] + denp[1]) + (denp[2] + denp[3]);
+        sX[hf * 128 + r] = (den0.x + den0.y) + (den1.x + den1.y);
         pair_sync(quarter);
         const float inv = 1.f / (z + (sX[r] + sX[128 + r]));
+        const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
         for (int c = 0; c < OD / 32; ++c) {
             float o[32];
             tmem_ld32f(trow + p.colO + hf * OD + 32 * c, o);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                uint4 u;
-                u.x = pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-                u.y = pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-                u.z = pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-                u.w = pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+                uint32_t uu[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 v = fmul2(make_float2(o[8 * q + 2 * i], o[8 * q + 2 * i + 1]), inv2);
+                    uu[i] = pack_bf16x2(v.x, v.y);
+                }
+                const uint4 u = make_uint4(uu[0], uu[1], uu[2], uu[3]);
                 *reinterpret_cast<uint4*>(sB2 + swz(r, hf * (OD / 8) + 4 * c + q)) = u;
             }
         }
