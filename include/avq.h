@@ -68,10 +68,11 @@ typedef enum {
     AVQ_ECUDA = -3,         /* a CUDA launch or runtime call failed */
     AVQ_ETIMEOUT = -4,      /* a bounded device-side wait ran out (reported by avq_device_status) */
     AVQ_EWORKSPACE = -5,    /* workspace missing or smaller than the *_workspace_bytes() answer */
-    AVQ_ERANGE = -6         /* (device status) for some query, a child's scaled logit exceeded the
-                               common shift of that query's weights (the largest non-empty parent
-                               logit, plus log n_p in the bf16 kernel) by more than 60 (natural-log
-                               units): its weights may overflow fp32 */
+    AVQ_ERANGE = -6         /* (device status, bf16 tensor-core kernel) for some query, a
+                               non-empty child's scaled logit plus log n_c exceeded the common
+                               shift of that query's weights (the largest non-empty parent logit
+                               plus log n_p) by more than 60 (natural-log units): its weights may
+                               overflow fp32 */
 } avq_status;
 
 /*
