@@ -102,40 +102,32 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
+// One butterfly level over 2H values: lanes with `up` keep the upper half and
+// send the lower one, the others the reverse; each kept value adds its
+// partner's (pairs of adds packed).
+template <int H>
+__device__ __forceinline__ void butterfly_level(float* v, bool up, int mask) {
+#pragma unroll
+    for (int j = 0; j < H; j += 2) {
+        const float k0 = up ? v[j + H] : v[j], s0 = up ? v[j] : v[j + H];
+        const float k1 = up ? v[j + 1 + H] : v[j + 1], s1 = up ? v[j + 1] : v[j + 1 + H];
+        const float r0 = __shfl_xor_sync(0xffffffffu, s0, mask);
+        const float r1 = __shfl_xor_sync(0xffffffffu, s1, mask);
+        const float2 o = fadd2(make_float2(k0, k1), make_float2(r0, r1));
+        v[j] = o.x;
+        v[j + 1] = o.y;
+    }
+}
+
 // Sum of each of 64 columns over the 32 lanes of a warp (a butterfly that
 // halves the number of values each step): on return lane L holds the sums of
 // columns 2L and 2L+1 in v[0], v[1].
 __device__ __forceinline__ void butterfly_colsum64(float* v, int lane) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const bool up = lane & 16;
-        const float keep = up ? v[j + 32] : v[j], send = up ? v[j] : v[j + 32];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const bool up = lane & 8;
-        const float keep = up ? v[j + 16] : v[j], send = up ? v[j] : v[j + 16];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const bool up = lane & 4;
-        const float keep = up ? v[j + 8] : v[j], send = up ? v[j] : v[j + 8];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const bool up = lane & 2;
-        const float keep = up ? v[j + 4] : v[j], send = up ? v[j] : v[j + 4];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const bool up = lane & 1;
-        const float keep = up ? v[j + 2] : v[j], send = up ? v[j] : v[j + 2];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-    }
+    butterfly_level<32>(v, lane & 16, 16);
+    butterfly_level<16>(v, lane & 8, 8);
+    butterfly_level<8>(v, lane & 4, 4);
+    butterfly_level<4>(v, lane & 2, 2);
+    butterfly_level<2>(v, lane & 1, 1);
 }
 
 // 32 TMEM columns of this warp's lanes into v (one wait for both loads).
@@ -178,8 +170,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     int* sRank = reinterpret_cast<int*>(sX + 256);           // [2][128] partial ranks
     unsigned long long* sKey = reinterpret_cast<unsigned long long*>(sRank + 256);   // [128]
     int* sSel = reinterpret_cast<int*>(sKey + 128);          // [128] selected parents
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + 128);   // q0, q1, mma, head
-    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + 128);   // q0, q1, mma, head, mma1
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 5);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r = tid & 127, hf = tid >> 7, quarter = warp & 3;
@@ -191,7 +183,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmO);
@@ -221,6 +213,20 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
         for (int kh = 0; kh < KH; ++kh)
             tma_load_3d(sQ0 + stage * IMG + kh * kRegion, &tmQ, &bars[stage], kh * 64, t * kTile, bh);
+    };
+    // (thread 0) MMA1 S_p = Q C_par^T of the tile whose Q is in stage `st`,
+    // completion on bars[4]; false if its Q never arrived
+    auto issue_mma1 = [&](int st) -> bool {
+        const bool okq = mbar_wait(&bars[st], (qph >> st) & 1u);
+        qph ^= 1u << st;
+        if (okq) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks)
+                mma_ss(tmem, desc_k(sQ0 + st * IMG, ks), desc_k(sB1, ks), idesc1, ks > 0);
+            mma_commit(&bars[4]);
+        }
+        return okq;
     };
     if (tid == 0 && g0 < g1) issue_q(g0, 0);
 
@@ -253,23 +259,19 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             cur_bh = bh;
         }
 
-        // ---- MMA1: S_p = Q C_par^T
+        // ---- MMA1: S_p = Q C_par^T (unless issued at the end of the previous
+        // tile), and the next tile's Q into the other stage
+        // (the next tile of the same (b,h) gets its MMA1 at the end of this one)
+        // (a tile issues the next one's MMA1 when that one is in the range and
+        // of the same (b,h); so this one's is issued here when it is the first
+        // of the range or of its (b,h))
         bool ok = true;
         if (tid == 0) {
-            ok = mbar_wait(&bars[stage], (qph >> stage) & 1u);
-            qph ^= 1u << stage;
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < KSTEPS; ++ks)
-                    mma_ss(tmem, desc_k(sQ0 + stage * IMG, ks), desc_k(sB1, ks), idesc1, ks > 0);
-                mma_commit(&bars[2]);
-                if (g + 1 < g1) issue_q(g + 1, stage ^ 1);
-            }
+            if (g == g0 || t == 0) ok = issue_mma1(stage);
+            if (ok && g + 1 < g1) issue_q(g + 1, stage ^ 1);
         }
         // (if thread 0 could not issue MMA1, every thread's wait below times out)
-        ok = mbar_wait(&bars[2], mphase) && ok;
-        mphase ^= 1;
+        ok = mbar_wait(&bars[4], (uint32_t)it & 1u) && ok;   // one MMA1 per tile, in order
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
 
@@ -486,6 +488,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 for (int ks = 0; ks < N2 / 16; ++ks)
                     mma_ts(tmem + p.colO, tmem + p.colWc + 8 * ks, desc_mn(sB3C, ks), idesc3, 1);
                 mma_commit(&bars[2]);
+                // every S column has been read: the next tile's MMA1 may write them
+                if (k == nchunks - 1 && g + 1 < g1 && t + 1 < p.ntiles) issue_mma1(stage ^ 1);
             }
             ok = mbar_wait(&bars[2], mphase);
             mphase ^= 1;
@@ -494,7 +498,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         if (failed) break;
         if (nchunks == 0) {   // P == 0: only the parents' contribution
-            if (tid == 0) mma_commit(&bars[2]);
+            if (tid == 0) {
+                mma_commit(&bars[2]);
+                if (g + 1 < g1 && t + 1 < p.ntiles) issue_mma1(stage ^ 1);
+            }
             ok = mbar_wait(&bars[2], mphase);
             mphase ^= 1;
             if (__syncthreads_or(!ok)) { failed = true; break; }
