@@ -259,12 +259,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             cur_bh = bh;
         }
 
-        // ---- MMA1: S_p = Q C_par^T (unless issued at the end of the previous
-        // tile), and the next tile's Q into the other stage
-        // (the next tile of the same (b,h) gets its MMA1 at the end of this one)
-        // (a tile issues the next one's MMA1 when that one is in the range and
-        // of the same (b,h); so this one's is issued here when it is the first
-        // of the range or of its (b,h))
+        // ---- MMA1: S_p = Q C_par^T, and the next tile's Q into the other stage.
+        // A tile issues the next one's MMA1 when that one is in the range and of
+        // the same (b,h); so this one's is issued here when it is the first of
+        // the range or of its (b,h). A failed wait (here and below) is acted on
+        // at the next CTA barrier, which every thread reaches.
         bool ok = true;
         if (tid == 0) {
             if (g == g0 || t == 0) ok = issue_mma1(stage);
@@ -272,7 +271,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         // (if thread 0 could not issue MMA1, every thread's wait below times out)
         ok = mbar_wait(&bars[4], (uint32_t)it & 1u) && ok;   // one MMA1 per tile, in order
-        if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
 
         // ---- parent pass over this half's 64 columns
@@ -343,7 +341,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             make_float2(x[0], x[1]);
         tmem_wait_st();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { failed = true; break; }
 
         // ---- importance and top-P selection: ranks over 64-bit keys, each
         // thread of a pair counting over half of the parents
@@ -364,7 +362,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 rk += (kk.x > key) + (kk.y > key);
             }
             sRank[hf * 128 + r] = rk;
-            __syncthreads();
+            pair_sync(quarter);   // the pair's two partial ranks
             if (tid < p.M0) {
                 const int rank = sRank[tid] + sRank[128 + tid];
                 if (rank < p.P) {
@@ -436,7 +434,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             cp_async_wait_all();
             fence_proxy_async_smem();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(!ok)) { failed = true; break; }
             if (tid == 0) {
                 tc_fence_after();
                 const uint32_t idesc2 = idesc_bf16_f32(128, N2, false);
@@ -445,9 +443,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     mma_ss(tmem + p.colSc, desc_k(sQ0 + stage * IMG, ks), desc_k(sB2, ks), idesc2, ks > 0);
                 mma_commit(&bars[2]);
             }
-            ok = mbar_wait(&bars[2], mphase);
+            ok = mbar_wait(&bars[2], mphase) && ok;
             mphase ^= 1;
-            if (__syncthreads_or(!ok)) { failed = true; break; }
             tc_fence_after();
 
             // child weights (A_c - A_p) n_c with A = 2^(sl2*S - m) for this half's
@@ -482,7 +479,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             tmem_wait_st();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(!ok)) { failed = true; break; }
             if (tid == 0) {
                 tc_fence_after();
                 for (int ks = 0; ks < N2 / 16; ++ks)
@@ -491,9 +488,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // every S column has been read: the next tile's MMA1 may write them
                 if (k == nchunks - 1 && g + 1 < g1 && t + 1 < p.ntiles) issue_mma1(stage ^ 1);
             }
-            ok = mbar_wait(&bars[2], mphase);
+            // (each thread's own wait also orders the next chunk's writes of
+            // the staging buffers and weight columns after this MMA3)
+            ok = mbar_wait(&bars[2], mphase) && ok;
             mphase ^= 1;
-            if (__syncthreads_or(!ok)) { failed = true; break; }
             tc_fence_after();
         }
         if (failed) break;
@@ -502,9 +500,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 mma_commit(&bars[2]);
                 if (g + 1 < g1 && t + 1 < p.ntiles) issue_mma1(stage ^ 1);
             }
-            ok = mbar_wait(&bars[2], mphase);
+            ok = mbar_wait(&bars[2], mphase) && ok;
             mphase ^= 1;
-            if (__syncthreads_or(!ok)) { failed = true; break; }
             tc_fence_after();
         }
 
@@ -531,7 +528,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { failed = true; break; }
         if (tid == 0) {
 #pragma unroll
             for (int kh = 0; kh < KH; ++kh) tma_store_3d(&tmO, sB2 + kh * kRegion, kh * 64, t * kTile, bh);
