@@ -81,7 +81,9 @@ const char* avq_status_string(int st) {
 
 size_t avq_precompute_workspace_bytes(const avq_shape* s) {
     if (check_shape(s) != AVQ_OK) return 0;
-    return kStatusBytes;
+    // status block, then room to list every key whose decision the fp32
+    // bounds leave open (8 bytes per key)
+    return kStatusBytes + align256(sizeof(long long) * (size_t)s->B * s->H * s->N);
 }
 
 int avq_precompute(const avq_shape* s, const void* K, const void* V, const void* codebook,
@@ -103,11 +105,14 @@ int avq_precompute(const avq_shape* s, const void* K, const void* V, const void*
     if (cudaMemsetAsync(vsum, 0, sizeof(float) * BH * Mtot * s->d, st) != cudaSuccess) return AVQ_ECUDA;
     if (s->N == 0) return AVQ_OK;
     cudaError_t e;
-    if (precompute_tc_supported(*s))
-        e = launch_precompute_tc(*s, K, V, codebook, assign, counts, vsum,
-                                 static_cast<StatusBlock*>(workspace), st);
-    else
+    if (precompute_tc_supported(*s)) {
+        // the open-key list starts empty (its length is status word 4)
+        StatusBlock* status = static_cast<StatusBlock*>(workspace);
+        if (cudaMemsetAsync(&status->pad[2], 0, sizeof(int32_t), st) != cudaSuccess) return AVQ_ECUDA;
+        e = launch_precompute_tc(*s, K, V, codebook, assign, counts, vsum, status, st);
+    } else {
         e = launch_precompute_simt(*s, K, V, codebook, assign, counts, vsum, st);
+    }
     return e == cudaSuccess ? AVQ_OK : AVQ_ECUDA;
 }
 

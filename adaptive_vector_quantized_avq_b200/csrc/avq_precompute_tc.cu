@@ -2,38 +2,36 @@
 // bf16 inputs (paper §4.2; papernotes, Key Designs 2; paper Table 1 rows
 // "VQ assignment" and "Value aggregation").
 //
-// Persistent: one 256-thread CTA per SM walks a contiguous range of 128-key
-// tiles (head-major). Key r of a tile is handled by the thread pair r and
-// r + 128 (halves h = 0, 1): each half holds half of the key's dimensions and
-// scans half of the parents. The pair combines its parent scans through shared
-// memory (both threads then hold the same nearest parent); for the children,
-// half 1 publishes its partial distances and half 0 completes them, decides
-// and writes the outputs. TMEM lane r holds key r's dot products.
+// Persistent: one CTA per SM walks a contiguous range of 128-key tiles
+// (head-major). The CTA runs independent 128-thread warpgroups (four at d=64,
+// two at d=128), one thread per key; warpgroup w takes tiles w, w+NWG, ... of
+// each (b,h) segment of the range, with its own K stage, TMEM accumulator and
+// mbarriers. The CTA meets only where the (b,h) changes.
 //
-// Per head (when the range enters it): TMA brings the parent codewords (the
-// B operand), cp.async brings the C*M0 child codewords into a shared-memory
+// Per head (when the range enters it): TMA brings the parent codewords (the B
+// operand), cp.async brings the C*M0 child codewords into a shared-memory
 // image whose 16-byte chunks are permuted by the parent index (so that keys
-// of different parents read different banks), and the parent norms
-// ||C_p||^2 are computed. Counts accumulate in shared memory and are flushed
-// with one global atomic per non-empty codeword when the head is done.
+// of different parents read different banks), and all codeword norms are
+// computed in fp64 and rounded once. Counts accumulate in shared memory and
+// are flushed with one global atomic per non-empty codeword.
 //
-// Per tile:
-//   1. TMA brings K and V (two stages, issued two tiles ahead).
-//   2. MMA  S = K C_par^T  (M=128, N=M0p, K=d) into one of two TMEM buffers,
-//      issued one tile ahead.
-//   3. a1: v_p = ||C_p||^2 - 2 S_p (the expanded distance minus ||k||^2) in
-//      fp32; the smallest and the runner-up. If they are not separated by the
-//      error bound of this expanded form, the parents within the band are
-//      re-decided with the exact fp64 distance summed in index order.
-//   4. a2: the kept parent and its C children by the direct form
-//      sum_j (k_j - c_j)^2 in fp32 (sm_100 mixed bf16/fp32 subtraction, so
-//      the codewords need no unpacking; relative error <= (d+4)u); a
-//      candidate wins only when strictly closer (parent first,
-//      lowest child index among equals); the band the bound cannot separate
-//      is re-decided in fp64.
-//   5. a3: assign written; counts in shared memory; the key's V row is added
-//      to the parent's and (when the key moved) the child's value sum with
-//      coalesced 16-byte fp32 vector reductions (one half-warp per row).
+// Per tile and warpgroup:
+//   1. TMA brings the K tile; MMA S = K C_par^T (M=128, N=M0p, K=d) into the
+//      warpgroup's TMEM columns.
+//   2. a1: v_p = ||C_p||^2 - 2 S_p (the expanded distance minus ||k||^2) in
+//      fp32: the minimum, then the parents within the error bound of this
+//      expanded form; more than one is re-decided with the exact fp64
+//      distance summed in index order.
+//   3. a2: the kept parent and its C children, v = ||C||^2 - 2 k.C with the
+//      dot product on CUDA cores (bf16 x bf16 mixed-precision fma, no
+//      unpacking) under a tighter bound; a child wins only when strictly
+//      closer (parent first, lowest child index among equals); the band the
+//      bound cannot separate is re-decided in fp64.
+//   4. a3: assign written; the key counts at its leaf (shared memory,
+//      warp-aggregated) and its V row (read from global memory, coalesced) is
+//      added to the leaf's value sum with 16-byte fp32 vector reductions.
+// A second kernel then adds each parent's children into the parent's totals,
+// so that a parent holds its whole cluster.
 #include <algorithm>
 
 #include "avq_internal.cuh"
@@ -56,6 +54,9 @@ struct TcPreParams {
     int32_t* counts;            // [BH, Mtot]
     float* vsum;                // [BH, Mtot, D]
     StatusBlock* status;
+    long long* fix_list;        // keys (b,h,n flattened) whose decision the fp32 bounds left open,
+                                // plus (nearest parent + 1) << 40 where only the leaf is open
+    int* fix_count;             // number of entries in fix_list (zeroed by the caller)
 };
 
 __device__ __forceinline__ uint8_t* align1024p(uint8_t* p) {
@@ -79,64 +80,6 @@ __device__ __forceinline__ uint32_t ch_off(int i, int p, int j) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// (c - k) for a bf16 c (low or high half of a 32-bit word) and an fp32 k,
-// rounded once (sm_100 mixed-precision subtraction; no unpacking)
-__device__ __forceinline__ float sub_lo(uint32_t w, float k) {
-    float r;
-    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tsub.rn.f32.bf16 %0, l, %2;\n\t}" : "=f"(r) : "r"(w), "f"(k));
-    return r;
-}
-__device__ __forceinline__ float sub_hi(uint32_t w, float k) {
-    float r;
-    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tsub.rn.f32.bf16 %0, h, %2;\n\t}" : "=f"(r) : "r"(w), "f"(k));
-    return r;
-}
-
-// Exact fp64 squared distance between two bf16 rows held in shared memory
-// (16-byte chunk j of each at xoff(j) / coff(j) from its base): terms
-// (x_j - c_j)^2 in index order, no fused operations, so that the sum is the
-// same double as a plain sequential fp64 loop over the row.
-template <int D, typename FX, typename FC>
-__device__ __noinline__ double exact_dist_smem(const uint8_t* xbase, FX xoff, const uint8_t* cbase, FC coff) {
-    double s = 0.0;
-#pragma unroll 1
-    for (int j = 0; j < D / 8; ++j) {
-        const uint4 xw = *reinterpret_cast<const uint4*>(xbase + xoff(j));
-        const uint4 cw = *reinterpret_cast<const uint4*>(cbase + coff(j));
-        const uint32_t xs[4] = {xw.x, xw.y, xw.z, xw.w}, cs[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const double x = (double)((e & 1) ? bf_hi(xs[e >> 1]) : bf_lo(xs[e >> 1]));
-            const double c = (double)((e & 1) ? bf_hi(cs[e >> 1]) : bf_lo(cs[e >> 1]));
-            const double t = __dsub_rn(x, c);
-            s = __dadd_rn(s, __dmul_rn(t, t));
-        }
-    }
-    return s;
-}
-// The same with the key's bf16 row in global memory (read once, all chunks
-// in flight together).
-template <int D, typename FC>
-__device__ __noinline__ double exact_dist_gk(const uint16_t* krow, const uint8_t* cbase, FC coff) {
-    uint4 kw[D / 8];
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) kw[j] = __ldg(reinterpret_cast<const uint4*>(krow) + j);
-    double s = 0.0;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-        const uint4 cw = *reinterpret_cast<const uint4*>(cbase + coff(j));
-        const uint32_t xs[4] = {kw[j].x, kw[j].y, kw[j].z, kw[j].w}, cs[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const double x = (double)((e & 1) ? bf_hi(xs[e >> 1]) : bf_lo(xs[e >> 1]));
-            const double c = (double)((e & 1) ? bf_hi(cs[e >> 1]) : bf_lo(cs[e >> 1]));
-            const double t = __dsub_rn(x, c);
-            s = __dadd_rn(s, __dmul_rn(t, t));
-        }
-    }
-    return s;
-}
-
 __device__ __forceinline__ void red_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
@@ -158,27 +101,6 @@ __device__ __forceinline__ bool wg_sync_or(int id, bool pred) {
     return r != 0;
 }
 
-// Squared distance of the key (fp32 registers) to a bf16 row in shared memory
-// whose 16-byte chunk j lives at chunk_off(j); each term (k - c)^2 rounded
-// once (fused), four independent accumulators.
-template <int D, typename F>
-__device__ __forceinline__ float full_dist(const float (&k)[D], const uint8_t* row_base, F chunk_off) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-        const uint4 w = *reinterpret_cast<const uint4*>(row_base + chunk_off(j));
-        const float t0 = sub_lo(w.x, k[8 * j + 0]), t1 = sub_hi(w.x, k[8 * j + 1]);
-        const float t2 = sub_lo(w.y, k[8 * j + 2]), t3 = sub_hi(w.y, k[8 * j + 3]);
-        const float t4 = sub_lo(w.z, k[8 * j + 4]), t5 = sub_hi(w.z, k[8 * j + 5]);
-        const float t6 = sub_lo(w.w, k[8 * j + 6]), t7 = sub_hi(w.w, k[8 * j + 7]);
-        a0 = __fmaf_rn(t0, t0, a0); a1 = __fmaf_rn(t1, t1, a1);
-        a2 = __fmaf_rn(t2, t2, a2); a3 = __fmaf_rn(t3, t3, a3);
-        a0 = __fmaf_rn(t4, t4, a0); a1 = __fmaf_rn(t5, t5, a1);
-        a2 = __fmaf_rn(t6, t6, a2); a3 = __fmaf_rn(t7, t7, a3);
-    }
-    return __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
-}
-
 // acc + x*x for the bf16 x in the low / high half of w, rounded once (sm_100
 // mixed-precision fma; x*x is exact in fp32, so this equals fmaf on the
 // widened value)
@@ -191,6 +113,62 @@ __device__ __forceinline__ float sqacc_hi(uint32_t w, float acc) {
     float r;
     asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, h, h, %2;\n\t}" : "=f"(r) : "r"(w), "f"(acc));
     return r;
+}
+
+// acc + x*c for the bf16 values in the low / high halves of kw and cw (the
+// product is exact in fp32; one rounding: sm_100 mixed-precision fma).
+__device__ __forceinline__ float dotacc_lo(uint32_t kw, uint32_t cw, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 kl, kh, cl, ch;\n\tmov.b32 {kl, kh}, %1;\n\tmov.b32 {cl, ch}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, kl, cl, %3;\n\t}" : "=f"(r) : "r"(kw), "r"(cw), "f"(acc));
+    return r;
+}
+__device__ __forceinline__ float dotacc_hi(uint32_t kw, uint32_t cw, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 kl, kh, cl, ch;\n\tmov.b32 {kl, kh}, %1;\n\tmov.b32 {cl, ch}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, kh, ch, %3;\n\t}" : "=f"(r) : "r"(kw), "r"(cw), "f"(acc));
+    return r;
+}
+// k . c for the key's packed bf16 row kw and a bf16 row in shared memory whose
+// 16-byte chunk j lives at chunk_off(j): sixteen accumulators of d/16 terms
+// each, combined pairwise, so the sum carries at most d/16 + 3 roundings.
+template <int D, typename F>
+__device__ __forceinline__ float dot_bf16(const uint4 (&kw)[D / 8], const uint8_t* row_base, F chunk_off) {
+    float a[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(row_base + chunk_off(j));
+        const int o = 8 * (j & 1);
+        a[o + 0] = dotacc_lo(kw[j].x, w.x, a[o + 0]); a[o + 1] = dotacc_hi(kw[j].x, w.x, a[o + 1]);
+        a[o + 2] = dotacc_lo(kw[j].y, w.y, a[o + 2]); a[o + 3] = dotacc_hi(kw[j].y, w.y, a[o + 3]);
+        a[o + 4] = dotacc_lo(kw[j].z, w.z, a[o + 4]); a[o + 5] = dotacc_hi(kw[j].z, w.z, a[o + 5]);
+        a[o + 6] = dotacc_lo(kw[j].w, w.w, a[o + 6]); a[o + 7] = dotacc_hi(kw[j].w, w.w, a[o + 7]);
+    }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) a[i] = __fadd_rn(a[i], a[i + w]);
+    return a[0];
+}
+// ||row||^2 of a bf16 row in shared memory, summed in fp64 and rounded once
+// to fp32 (error <= 2^-24 relative, to within fp64 rounding).
+template <int D, typename F>
+__device__ __forceinline__ float norm2_f64(const uint8_t* row_base, F chunk_off) {
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(row_base + chunk_off(j));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double lo = (double)bf_lo(ww[e]), hi = (double)bf_hi(ww[e]);
+            s = __fma_rn(lo, lo, s);
+            s = __fma_rn(hi, hi, s);
+        }
+    }
+    return __double2float_rn(s);
 }
 
 // Three-input fp32 minimum (sm_100).
@@ -220,9 +198,10 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     const uint32_t b1_region = (uint32_t)p.M0p * 128u;   // bytes between its 64-column blocks
     uint8_t* sCh = sB1 + KH * b1_region;           // children image [M0*C rows x D] bf16
     const size_t ch_bytes = (size_t)p.M0 * C * D * 2;
-    float* sCn = reinterpret_cast<float*>(sCh + ((ch_bytes + 15) & ~size_t(15)));   // [128]
-    float* sRed = sCn + 128;                       // [4]
-    int* sCnt = reinterpret_cast<int*>(sRed + 4);  // [Mtot]
+    float* sCn = reinterpret_cast<float*>(sCh + ((ch_bytes + 15) & ~size_t(15)));   // [128] parent norms
+    float* sRed = sCn + 128;                       // [16]
+    float* sCcn = sRed + 16;                       // [M0*C] child norms
+    int* sCnt = reinterpret_cast<int*>(sCcn + p.M0 * C);   // [Mtot]
     uint64_t* bars = reinterpret_cast<uint64_t*>(
         (reinterpret_cast<uintptr_t>(sCnt + p.Mtot) + 7) & ~uintptr_t(7));
     // bars: per warpgroup w: 2w = K stage, 2w+1 = MMA; 2*NWG = head
@@ -255,7 +234,6 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     const uint32_t tmem = *sTmem;
     const uint32_t trow = tmem + 128 * wg + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t idesc = idesc_bf16_f32(128, p.M0p, false);
-    const float eps_dir = dist_eps(D);
     // expanded-form bound factor: 2 * (5d + 8) * 2^-24 (per distance, times
     // ||k||^2 + max ||C_p||^2)
     const float c_exp = 2.f * (5.f * D + 8.f) * 5.9604644775390625e-08f;
@@ -287,6 +265,9 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         const int bh = gs / p.ntiles, h = bh % p.H;
         const int ge = min(g1, (bh + 1) * p.ntiles);
         __syncthreads();   // every warpgroup is done with the previous segment
+        // this warpgroup's first K tile of the segment (its stage is free; the
+        // load overlaps the head data below)
+        if (lt == 0 && gs + wg < ge) issue_k(gs + wg);
         if (cur_bh >= 0) flush_counts(cur_bh);
         bool ok = true;
         if (cur_bh < 0 || h != cur_bh % p.H) {
@@ -303,36 +284,36 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             cp_async_commit();
             ok = mbar_wait(barH, hph);
             hph ^= 1;
-            // ||C_p||^2 from the parent image, terms in index order; +inf for
-            // padding parents (p >= M0): they never win
-            if (tid < 128) {
-                float cn = 0.f;
-                if (tid < p.M0 && ok) {
-#pragma unroll
-                    for (int j = 0; j < D / 8; ++j) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(sB1 + swz_off(tid, j, b1_region));
-                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            cn = __fmaf_rn(bf_lo(ww[e]), bf_lo(ww[e]), cn);
-                            cn = __fmaf_rn(bf_hi(ww[e]), bf_hi(ww[e]), cn);
-                        }
-                    }
-                }
-                sCn[tid] = tid < p.M0 ? cn : INFINITY;
-                float mx = cn;
-#pragma unroll
-                for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                if (lane == 0) sRed[warp] = mx;
-            }
+            // codeword norms ||C||^2 (fp64, rounded once); +inf for padding
+            // parents (p >= M0): they never win. The bounds below use the
+            // largest norm of the head's parents and children.
             cp_async_wait_all();
+            __syncthreads();   // the children image is complete
+            float mx = 0.f;
+            if (tid < 128) {
+                float cn = INFINITY;
+                if (tid < p.M0 && ok) {
+                    cn = norm2_f64<D>(sB1, [&](int j) { return swz_off(tid, j, b1_region); });
+                    mx = cn;
+                }
+                sCn[tid] = cn;
+            }
+            for (int i = tid; i < p.M0 * C; i += NT) {
+                const float cn = norm2_f64<D>(sCh, [&](int j) { return ch_off<D>(i, i / C, j); });
+                sCcn[i] = cn;
+                mx = fmaxf(mx, cn);
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) sRed[warp] = mx;
         }
         if (__syncthreads_or(!ok)) { failed = true; break; }
-        cnmax = fmaxf(fmaxf(sRed[0], sRed[1]), fmaxf(sRed[2], sRed[3]));
+        cnmax = sRed[0];
+#pragma unroll
+        for (int w = 1; w < NT / 32; ++w) cnmax = fmaxf(cnmax, sRed[w]);
         cur_bh = bh;
 
         // this warpgroup's tiles of the segment
-        if (lt == 0 && gs + wg < ge) issue_k(gs + wg);
         for (int g = gs + wg; g < ge; g += NWG) {
             const int t = g % p.ntiles;
             const int rows = min(kTile, p.N - t * kTile);
@@ -413,90 +394,50 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                     }
                 }
             }
+            // more than one parent in the band: decided later in fp64 (the key
+            // is listed; parent 0 stands in until then)
             int bp = (acc & 255) == 1 ? (acc >> 8) : 0;
-            const bool redecide = valid && (acc & 255) != 1;
-            if (__any_sync(0xffffffffu, redecide)) {
-                // exact fp64 distances of the parents within the band, in
-                // index order (TMEM reloads are warp-wide, the fp64 work only
-                // where needed)
-                double eb = INFINITY;
-                int ep = 0;
-                for (int c = 0; c < p.M0p; c += 16) {
-                    float v16[16];
-                    tmem_ld16f(trow + c, v16);
-                    tmem_wait_ld();
-                    tmem_touch16f(v16);
-                    if (redecide) {
-                        for (int q = 0; q < 16; ++q) {
-                            const int pp = c + q;
-                            if (pp >= p.M0) break;
-                            if (!(fmaf(-2.f, v16[q], sCn[pp]) <= thr)) continue;
-                            const double e = exact_dist_smem<D>(
-                                sK, [&](int j) { return swz_off(lt, j); }, sB1,
-                                [&](int j) { return swz_off(pp, j, b1_region); });
-                            if (e < eb) { eb = e; ep = pp; }
-                        }
-                    }
-                }
-                if (redecide) {
-                    bp = ep;
-                    ++n_pre;
-                }
-            }
-            // key row -> fp32 registers
-            float k[D];
+            bool listed = valid && (acc & 255) != 1;
+            n_pre += listed;
+            // key row (packed bf16) -> registers
+            uint4 kw[D / 8];
 #pragma unroll
-            for (int j = 0; j < D / 8; ++j) {
-                const uint4 w = *reinterpret_cast<const uint4*>(sK + swz_off(lt, j));
-                k[8 * j + 0] = bf_lo(w.x); k[8 * j + 1] = bf_hi(w.x);
-                k[8 * j + 2] = bf_lo(w.y); k[8 * j + 3] = bf_hi(w.y);
-                k[8 * j + 4] = bf_lo(w.z); k[8 * j + 5] = bf_hi(w.z);
-                k[8 * j + 6] = bf_lo(w.w); k[8 * j + 7] = bf_hi(w.w);
-            }
+            for (int j = 0; j < D / 8; ++j) kw[j] = *reinterpret_cast<const uint4*>(sK + swz_off(lt, j));
             tc_fence_before();   // this tile's TMEM reads before the next MMA into the buffer
             if (wg_sync_or(wgbar, !ok)) { failed = true; break; }   // also: the K stage is free
             if (lt == 0 && g + NWG < ge) issue_k(g + NWG);
 
-            // ---- a2: the kept parent and its children, direct form. A child
-            // wins only when strictly closer (parent first, lowest child index
-            // among equals); the runner-up decides whether the bound separates
-            // the winner from every other candidate (the test is monotone in
-            // the runner-up's distance).
+            // ---- a2: the kept parent and its children, v = ||C||^2 - 2 k.C with
+            // the dot product on CUDA cores (bf16 x bf16 products exact, d/16 + 3
+            // roundings) and fp64-rounded norms: |error| <= (d/16 + 5.5) u
+            // (||k||^2 + max ||C||^2), bounded here by Ec. A child wins only when
+            // strictly closer (parent first, lowest child index among equals);
+            // the winner is certain when the runner-up lies more than 2 Ec above
+            // it, else the key is listed for the fp64 decision.
             int leaf = bp;
             {
-                const float dpar = full_dist<D>(k, sB1, [&](int j) { return swz_off(bp, j, b1_region); });
-                float lo = dpar, sec = INFINITY;
+                const float Ec = (0.0625f * D + 7.f) * 1.0625f * 5.9604644775390625e-08f * (kn + cnmax);
+                float lo = fmaf(-2.f, dot_bf16<D>(kw, sB1, [&](int j) { return swz_off(bp, j, b1_region); }),
+                                sCn[bp]);
+                float sec = INFINITY;
                 int lo_i = -1;
 #pragma unroll
                 for (int c = 0; c < C; ++c) {
                     const int i = bp * C + c;
-                    const float dc = full_dist<D>(k, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
-                    if (dc < lo) { sec = lo; lo = dc; lo_i = c; }
-                    else sec = fminf(sec, dc);
+                    const float vc =
+                        fmaf(-2.f, dot_bf16<D>(kw, sCh, [&](int j) { return ch_off<D>(i, bp, j); }), sCcn[i]);
+                    if (vc < lo) { sec = lo; lo = vc; lo_i = c; }
+                    else sec = fminf(sec, vc);
                 }
-                if (separated(lo, sec, eps_dir) || !valid) {
-                    leaf = lo_i < 0 ? bp : p.M0 + bp * C + lo_i;
-                } else {
-                    // fp64 among the parent and the children within the band
-                    // (the key row comes back from global memory: its stage
-                    // may already hold the next tile)
-                    uint32_t band = 0;
-                    for (int c = 0; c < C; ++c) {
-                        const int i = bp * C + c;
-                        const float dc = full_dist<D>(k, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
-                        if (!separated(lo, dc, eps_dir)) band |= 1u << c;
-                    }
-                    const uint16_t* krow = p.K + ((size_t)bh * p.N + (size_t)t * kTile + lt) * D;
-                    double eb = exact_dist_gk<D>(krow, sB1, [&](int j) { return swz_off(bp, j, b1_region); });
-                    int win = bp;
-                    for (; band; band &= band - 1) {
-                        const int i = bp * C + __ffs(band) - 1;
-                        const double e = exact_dist_gk<D>(krow, sCh, [&](int j) { return ch_off<D>(i, bp, j); });
-                        if (e < eb) { eb = e; win = p.M0 + i; }
-                    }
-                    leaf = win;
-                    ++n_chd;
-                }
+                leaf = lo_i < 0 ? bp : p.M0 + bp * C + lo_i;
+                const bool open = valid && !(sec - lo > 2.f * Ec);
+                n_chd += open;
+                listed = listed || open;
+            }
+            if (listed) {
+                const int slot = atomicAdd(p.fix_count, 1);
+                const long long kidx = (long long)bh * p.N + (long long)t * kTile + lt;
+                p.fix_list[slot] = (acc & 255) == 1 ? kidx | ((long long)(bp + 1) << 40) : kidx;
             }
 
             // ---- a3: outputs. Counts and value sums go to the leaf only (the
@@ -571,6 +512,105 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     }
 }
 
+// Exact fp64 squared distance between the key (its bf16 row in registers,
+// eight values per 16-byte word) and a bf16 row in global memory (read as
+// 16-byte words), terms (x_j - c_j)^2 in index order with no fused operations:
+// the same double as a plain sequential fp64 loop over the row.
+template <int D>
+__device__ __forceinline__ double exact_dist_rows(const uint4 (&kw)[D / 8], const uint16_t* c) {
+    uint4 cw[D / 8];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) cw[j] = __ldg(reinterpret_cast<const uint4*>(c) + j);
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+        const uint32_t xs[4] = {kw[j].x, kw[j].y, kw[j].z, kw[j].w}, cs[4] = {cw[j].x, cw[j].y, cw[j].z, cw[j].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double xv = (double)((e & 1) ? bf_hi(xs[e >> 1]) : bf_lo(xs[e >> 1]));
+            const double cv = (double)((e & 1) ? bf_hi(cs[e >> 1]) : bf_lo(cs[e >> 1]));
+            const double t = __dsub_rn(xv, cv);
+            s = __dadd_rn(s, __dmul_rn(t, t));
+        }
+    }
+    return s;
+}
+
+// (distance, index) minimum over a warp, the lower index among equal distances.
+__device__ __forceinline__ void warp_argmin(double& d, int& i) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const double od = __shfl_xor_sync(0xffffffffu, d, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+        if (od < d || (od == d && oi < i)) { d = od; i = oi; }
+    }
+}
+
+// The exact decision for the listed keys (one 128-thread block per key): the
+// nearest parent (one thread per parent) unless the entry carries it, then
+// the leaf from the parent's and its children's distances (one thread each),
+// all fp64 summed in index order, with the tie rules of the main kernel. Where
+// the provisional leaf differs, the key's count and V row move from it to the
+// exact leaf (before the parents' totals are formed).
+template <int D, int C>
+__global__ void __launch_bounds__(128) precompute_fixup_kernel(const TcPreParams p, const uint16_t* V) {
+    __shared__ double sD[4];
+    __shared__ int sI[4];
+    const int n_fix = *p.fix_count;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = blockIdx.x; e < n_fix; e += gridDim.x) {
+        const long long entry = p.fix_list[e];
+        const long long key = entry & ((1LL << 40) - 1);
+        int bp = (int)(entry >> 40) - 1;   // -1: the parent is open too
+        const long long bh = key / p.N;
+        const int h = (int)(bh % p.H);
+        uint4 kw[D / 8];
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) kw[j] = __ldg(reinterpret_cast<const uint4*>(p.K + key * D) + j);
+        const uint16_t* cbh = p.codebook + (size_t)h * p.Mtot * D;
+        if (bp < 0) {
+            double dp = INFINITY;
+            int ip = p.M0;
+            if (tid < p.M0) {
+                dp = exact_dist_rows<D>(kw, cbh + (size_t)tid * D);
+                ip = tid;
+            }
+            warp_argmin(dp, ip);
+            if (lane == 0) { sD[warp] = dp; sI[warp] = ip; }
+            __syncthreads();
+            dp = lane < 4 ? sD[lane] : INFINITY;
+            ip = lane < 4 ? sI[lane] : p.M0;
+            warp_argmin(dp, ip);
+            bp = ip < p.M0 ? ip : 0;   // (ip == M0 only for non-finite inputs)
+        }
+        if (warp == 0) {
+            // lanes 0..C-1: the children; lane C: the parent
+            double d = INFINITY;
+            if (lane <= C) d = exact_dist_rows<D>(kw, cbh + (size_t)(lane < C ? p.M0 + bp * C + lane : bp) * D);
+            const double dpar = __shfl_sync(0xffffffffu, d, C);
+            int cc = lane < C ? lane : C;
+            if (lane >= C) d = INFINITY;
+            warp_argmin(d, cc);
+            const int leaf = d < dpar ? p.M0 + bp * C + cc : bp;
+            const int old = p.assign[key];
+            if (old != leaf) {
+                const size_t base = (size_t)bh * p.Mtot;
+                if (lane == 0) {
+                    p.assign[key] = leaf;
+                    atomicSub(p.counts + base + old, 1);
+                    atomicAdd(p.counts + base + leaf, 1);
+                }
+                for (int j = lane; j < D; j += 32) {
+                    const float v = __uint_as_float((uint32_t)__ldg(V + key * D + j) << 16);
+                    atomicAdd(p.vsum + (base + old) * D + j, -v);
+                    atomicAdd(p.vsum + (base + leaf) * D + j, v);
+                }
+            }
+        }
+        __syncthreads();   // sD/sI are rewritten for the next key
+    }
+}
+
 // Completes the parents' totals: counts[p] and vsum[p] (which so far hold the
 // keys that stayed at the parent) plus those of the parent's C children. One
 // warp per (b, h, parent).
@@ -604,7 +644,8 @@ size_t pre_smem_bytes(int D, int M0, int C, int Mtot) {
     const int nwg = pre_nwg(D);
     const size_t M0p = (size_t)((M0 + 15) & ~15);
     return 1024 + nwg * (size_t)(D / 64) * kRegion + (size_t)(D / 64) * M0p * 128 +
-           (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) + 128 * 4 /*sCn*/ + 4 * 4 /*sRed*/ + (size_t)Mtot * 4 +
+           (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) + 128 * 4 /*sCn*/ + 16 * 4 /*sRed*/ +
+           (size_t)M0 * C * 4 /*sCcn*/ + (size_t)Mtot * 4 +
            8 + (2 * nwg + 1) * 8 + 16;
 }
 
@@ -634,6 +675,9 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     prm.counts = counts;
     prm.vsum = vsum;
     prm.status = status;
+    // the workspace holds the status block, then the list of open keys
+    prm.fix_count = &status->pad[2];
+    prm.fix_list = reinterpret_cast<long long*>(reinterpret_cast<uint8_t*>(status) + kStatusBytes);
     const size_t smem = pre_smem_bytes(D, s.M0, C, Mtot);
     constexpr int NWG = D == 64 ? 4 : 2;
     auto kern = precompute_tc_kernel<D, C, NWG>;
@@ -644,6 +688,10 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = std::min(prm.total_tiles, sms);
     kern<<<grid, 128 * NWG, smem, st>>>(tk, tcb, prm);
+    count_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    precompute_fixup_kernel<D, C><<<sms * 16, 128, 0, st>>>(prm, static_cast<const uint16_t*>(V));
     count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -305,6 +305,12 @@ def run_ours(args):
     att_ms = [e[1].elapsed_time(e[2]) for e in evs]
     if bd.avq_device_status(ws_pre, sp) or bd.avq_device_status(ws_att, sp):
         raise RuntimeError("device status error after timing")
+    # keys whose parent / leaf the fp32 bounds could not certify, re-decided in
+    # fp64 by the precompute kernel (counters in its status block, summed over
+    # the warm-up and timed calls)
+    diag = ws_pre[:16].view(torch.int32).cpu().tolist()
+    ncalls = args.warmup + args.steps
+    redecided = [diag[2] / ncalls, diag[3] / ncalls]
 
     # end to end through the public API: pinned host inputs in, output out
     hK, hV, hQ, hcb = (pinned(getattr(inp, n)) for n in ("K", "V", "Q", "codebook"))
@@ -364,6 +370,7 @@ def run_ours(args):
                        "seed": f"{wl.seed}+rank"},
             "kernels": {k: {"ms_avg": kern[k], "ms_min": min(pre_ms if k == 'precompute' else att_ms),
                             "roofline": rl[k]} for k in kern},
+            "fp64_redecided_per_call": {"parent": redecided[0], "leaf": redecided[1]},
             "roofline": roof,
             "clocks": clk,
             "e2e": {"value": rows_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

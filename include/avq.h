@@ -77,8 +77,10 @@ typedef enum {
 
 /*
  * Workspace needed by avq_precompute for `s` (bytes, a multiple of 256;
- * 0 for invalid shapes). The workspace holds the device status word read by
- * avq_device_status and per-head scratch of the aggregation.
+ * 0 for invalid shapes): 256 bytes for the device status word read by
+ * avq_device_status, then 8 bytes per key (B*H*N) for the list of keys whose
+ * nearest parent or leaf the kernel's fp32 error bounds leave open; those keys
+ * are decided exactly (fp64) by a second pass of the same call.
  */
 size_t avq_precompute_workspace_bytes(const avq_shape* s);
 
