@@ -5,6 +5,8 @@
 
 #include <atomic>
 
+#include <algorithm>
+
 #include "avq_internal.cuh"
 
 namespace avq {
@@ -79,11 +81,24 @@ const char* avq_status_string(int st) {
     }
 }
 
+namespace {
+// Zeroes the precompute outputs that are accumulated (counts, vsum): one
+// launch instead of two memsets.
+__global__ void zero_accumulators_kernel(int32_t* counts, size_t n_counts, float4* vsum4, size_t n_vsum4) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (size_t i = i0; i < n_vsum4; i += stride) vsum4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (size_t i = i0; i < n_counts; i += stride) counts[i] = 0;
+}
+}  // namespace
+
 size_t avq_precompute_workspace_bytes(const avq_shape* s) {
     if (check_shape(s) != AVQ_OK) return 0;
     // status block, then room to list every key whose decision the fp32
-    // bounds leave open (8 bytes per key)
-    return kStatusBytes + align256(sizeof(long long) * (size_t)s->B * s->H * s->N);
+    // bounds leave open: 8 bytes per key, the last 128-key tile of each
+    // sequence counted whole
+    const size_t tiles = (size_t)s->B * s->H * (((size_t)s->N + 127) / 128);
+    return kStatusBytes + align256(sizeof(long long) * tiles * 128);
 }
 
 int avq_precompute(const avq_shape* s, const void* K, const void* V, const void* codebook,
@@ -101,14 +116,20 @@ int avq_precompute(const avq_shape* s, const void* K, const void* V, const void*
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t Mtot = (size_t)s->M0 * (1 + s->C);
     const size_t BH = (size_t)s->B * s->H;
-    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * BH * Mtot, st) != cudaSuccess) return AVQ_ECUDA;
-    if (cudaMemsetAsync(vsum, 0, sizeof(float) * BH * Mtot * s->d, st) != cudaSuccess) return AVQ_ECUDA;
+    const bool tc = s->N > 0 && precompute_tc_supported(*s);
+    StatusBlock* status = static_cast<StatusBlock*>(workspace);
+    {
+        // counts and vsum start at zero
+        const size_t n4 = BH * Mtot * s->d / 4;   // d is a multiple of 4
+        const unsigned blocks = (unsigned)std::min<size_t>((n4 + 255) / 256, 1024);
+        zero_accumulators_kernel<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(
+            counts, BH * Mtot, reinterpret_cast<float4*>(vsum), n4);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return AVQ_ECUDA;
+    }
     if (s->N == 0) return AVQ_OK;
     cudaError_t e;
-    if (precompute_tc_supported(*s)) {
-        // the open-key list starts empty (its length is status word 4)
-        StatusBlock* status = static_cast<StatusBlock*>(workspace);
-        if (cudaMemsetAsync(&status->pad[2], 0, sizeof(int32_t), st) != cudaSuccess) return AVQ_ECUDA;
+    if (tc) {
         e = launch_precompute_tc(*s, K, V, codebook, assign, counts, vsum, status, st);
     } else {
         e = launch_precompute_simt(*s, K, V, codebook, assign, counts, vsum, st);

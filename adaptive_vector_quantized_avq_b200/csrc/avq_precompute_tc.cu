@@ -55,8 +55,8 @@ struct TcPreParams {
     float* vsum;                // [BH, Mtot, D]
     StatusBlock* status;
     long long* fix_list;        // keys (b,h,n flattened) whose decision the fp32 bounds left open,
-                                // plus (nearest parent + 1) << 40 where only the leaf is open
-    int* fix_count;             // number of entries in fix_list (zeroed by the caller)
+                                // plus (nearest parent + 1) << 40 where only the leaf is open;
+                                // the CTA with tiles [g0, g1) owns entries [128 g0, 128 g1)
 };
 
 __device__ __forceinline__ uint8_t* align1024p(uint8_t* p) {
@@ -171,6 +171,92 @@ __device__ __forceinline__ float norm2_f64(const uint8_t* row_base, F chunk_off)
     return __double2float_rn(s);
 }
 
+// Exact fp64 squared distance between the key (its bf16 row in registers,
+// eight values per 16-byte word) and a bf16 row in global memory (read as
+// 16-byte words), terms (x_j - c_j)^2 in index order with no fused operations:
+// the same double as a plain sequential fp64 loop over the row.
+template <int D>
+__device__ __forceinline__ double exact_dist_rows(const uint4 (&kw)[D / 8], const uint16_t* c) {
+    uint4 cw[D / 8];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) cw[j] = __ldg(reinterpret_cast<const uint4*>(c) + j);
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+        const uint32_t xs[4] = {kw[j].x, kw[j].y, kw[j].z, kw[j].w}, cs[4] = {cw[j].x, cw[j].y, cw[j].z, cw[j].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double xv = (double)((e & 1) ? bf_hi(xs[e >> 1]) : bf_lo(xs[e >> 1]));
+            const double cv = (double)((e & 1) ? bf_hi(cs[e >> 1]) : bf_lo(cs[e >> 1]));
+            const double t = __dsub_rn(xv, cv);
+            s = __dadd_rn(s, __dmul_rn(t, t));
+        }
+    }
+    return s;
+}
+
+// (distance, index) minimum over a warp, the lower index among equal distances.
+__device__ __forceinline__ void warp_argmin(double& d, int& i) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const double od = __shfl_xor_sync(0xffffffffu, d, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+        if (od < d || (od == d && oi < i)) { d = od; i = oi; }
+    }
+}
+
+// The exact decision for one listed key (called by a whole warp): the nearest
+// parent (lanes over the parents) unless the entry carries it, then the leaf
+// from the parent's and its children's distances (one lane each), all fp64
+// summed in index order, with the tie rules of the main loop. Where the
+// provisional leaf differs, the key's count and V row move from it to the
+// exact leaf. Not inlined: the main loop keeps its registers.
+template <int D, int C>
+__device__ __noinline__ void fix_key(long long entry, const uint16_t* K, const uint16_t* V, const uint16_t* codebook,
+                                     int32_t* assign, int32_t* counts, float* vsum, int N, int H, int M0, int Mtot) {
+    const int lane = threadIdx.x & 31;
+    const long long key = entry & ((1LL << 40) - 1);
+    int bp = (int)(entry >> 40) - 1;   // -1: the parent is open too
+    const long long bh = key / N;
+    const int h = (int)(bh % H);
+    uint4 kw[D / 8];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) kw[j] = __ldg(reinterpret_cast<const uint4*>(K + key * D) + j);
+    const uint16_t* cbh = codebook + (size_t)h * Mtot * D;
+    if (bp < 0) {
+        double dp = INFINITY;
+        int ip = M0;
+        for (int pp = lane; pp < M0; pp += 32) {
+            const double d = exact_dist_rows<D>(kw, cbh + (size_t)pp * D);
+            if (d < dp) { dp = d; ip = pp; }
+        }
+        warp_argmin(dp, ip);
+        bp = ip < M0 ? ip : 0;   // (ip == M0 only for non-finite inputs)
+    }
+    // lanes 0..C-1: the children; lane C: the parent
+    double d = INFINITY;
+    if (lane <= C) d = exact_dist_rows<D>(kw, cbh + (size_t)(lane < C ? M0 + bp * C + lane : bp) * D);
+    const double dpar = __shfl_sync(0xffffffffu, d, C);
+    int cc = lane < C ? lane : C;
+    if (lane >= C) d = INFINITY;
+    warp_argmin(d, cc);
+    const int leaf = d < dpar ? M0 + bp * C + cc : bp;
+    const int old = assign[key];
+    if (old != leaf) {
+        const size_t base = (size_t)bh * Mtot;
+        if (lane == 0) {
+            assign[key] = leaf;
+            atomicSub(counts + base + old, 1);
+            atomicAdd(counts + base + leaf, 1);
+        }
+        for (int j = lane; j < D; j += 32) {
+            const float v = __uint_as_float((uint32_t)__ldg(V + key * D + j) << 16);
+            atomicAdd(vsum + (base + old) * D + j, -v);
+            atomicAdd(vsum + (base + leaf) * D + j, v);
+        }
+    }
+}
+
 // Three-input fp32 minimum (sm_100).
 __device__ __forceinline__ float fmin3(float a, float b, float c) {
     float r;
@@ -202,8 +288,9 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     float* sRed = sCn + 128;                       // [16]
     float* sCcn = sRed + 16;                       // [M0*C] child norms
     int* sCnt = reinterpret_cast<int*>(sCcn + p.M0 * C);   // [Mtot]
+    int* sFix = sCnt + p.Mtot;                             // [1] entries this CTA listed
     uint64_t* bars = reinterpret_cast<uint64_t*>(
-        (reinterpret_cast<uintptr_t>(sCnt + p.Mtot) + 7) & ~uintptr_t(7));
+        (reinterpret_cast<uintptr_t>(sFix + 1) + 7) & ~uintptr_t(7));
     // bars: per warpgroup w: 2w = K stage, 2w+1 = MMA; 2*NWG = head
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 2 * NWG + 1);
 
@@ -222,6 +309,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         tmem_relinquish();
     }
     if (tid == 0) {
+        *sFix = 0;
         for (int i = 0; i < 2 * NWG + 1; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmK);
@@ -435,9 +523,9 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                 listed = listed || open;
             }
             if (listed) {
-                const int slot = atomicAdd(p.fix_count, 1);
+                const int slot = atomicAdd(sFix, 1);
                 const long long kidx = (long long)bh * p.N + (long long)t * kTile + lt;
-                p.fix_list[slot] = (acc & 255) == 1 ? kidx | ((long long)(bp + 1) << 40) : kidx;
+                p.fix_list[(size_t)g0 * kTile + slot] = (acc & 255) == 1 ? kidx | ((long long)(bp + 1) << 40) : kidx;
             }
 
             // ---- a3: outputs. Counts and value sums go to the leaf only (the
@@ -498,6 +586,14 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 
     __syncthreads();
     if (!failed && cur_bh >= 0) flush_counts(cur_bh);
+    // the exact decisions for the keys this CTA listed (one warp per key;
+    // counts and sums are moved with global atomics, after the flush)
+    if (!failed) {
+        const int nf = *sFix;
+        for (int e = warp; e < nf; e += NT / 32)
+            fix_key<D, C>(p.fix_list[(size_t)g0 * kTile + e], p.K, p.V, p.codebook, p.assign, p.counts, p.vsum, p.N,
+                          p.H, p.M0, p.Mtot);
+    }
     if (failed && tid == 0) {
         atomicExch(&p.status->error, (int)AVQ_ETIMEOUT);
         atomicExch(&p.status->where, (int)blockIdx.x);
@@ -509,105 +605,6 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 128 * NWG);
-    }
-}
-
-// Exact fp64 squared distance between the key (its bf16 row in registers,
-// eight values per 16-byte word) and a bf16 row in global memory (read as
-// 16-byte words), terms (x_j - c_j)^2 in index order with no fused operations:
-// the same double as a plain sequential fp64 loop over the row.
-template <int D>
-__device__ __forceinline__ double exact_dist_rows(const uint4 (&kw)[D / 8], const uint16_t* c) {
-    uint4 cw[D / 8];
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) cw[j] = __ldg(reinterpret_cast<const uint4*>(c) + j);
-    double s = 0.0;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-        const uint32_t xs[4] = {kw[j].x, kw[j].y, kw[j].z, kw[j].w}, cs[4] = {cw[j].x, cw[j].y, cw[j].z, cw[j].w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const double xv = (double)((e & 1) ? bf_hi(xs[e >> 1]) : bf_lo(xs[e >> 1]));
-            const double cv = (double)((e & 1) ? bf_hi(cs[e >> 1]) : bf_lo(cs[e >> 1]));
-            const double t = __dsub_rn(xv, cv);
-            s = __dadd_rn(s, __dmul_rn(t, t));
-        }
-    }
-    return s;
-}
-
-// (distance, index) minimum over a warp, the lower index among equal distances.
-__device__ __forceinline__ void warp_argmin(double& d, int& i) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        const double od = __shfl_xor_sync(0xffffffffu, d, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-        if (od < d || (od == d && oi < i)) { d = od; i = oi; }
-    }
-}
-
-// The exact decision for the listed keys (one 128-thread block per key): the
-// nearest parent (one thread per parent) unless the entry carries it, then
-// the leaf from the parent's and its children's distances (one thread each),
-// all fp64 summed in index order, with the tie rules of the main kernel. Where
-// the provisional leaf differs, the key's count and V row move from it to the
-// exact leaf (before the parents' totals are formed).
-template <int D, int C>
-__global__ void __launch_bounds__(128) precompute_fixup_kernel(const TcPreParams p, const uint16_t* V) {
-    __shared__ double sD[4];
-    __shared__ int sI[4];
-    const int n_fix = *p.fix_count;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int e = blockIdx.x; e < n_fix; e += gridDim.x) {
-        const long long entry = p.fix_list[e];
-        const long long key = entry & ((1LL << 40) - 1);
-        int bp = (int)(entry >> 40) - 1;   // -1: the parent is open too
-        const long long bh = key / p.N;
-        const int h = (int)(bh % p.H);
-        uint4 kw[D / 8];
-#pragma unroll
-        for (int j = 0; j < D / 8; ++j) kw[j] = __ldg(reinterpret_cast<const uint4*>(p.K + key * D) + j);
-        const uint16_t* cbh = p.codebook + (size_t)h * p.Mtot * D;
-        if (bp < 0) {
-            double dp = INFINITY;
-            int ip = p.M0;
-            if (tid < p.M0) {
-                dp = exact_dist_rows<D>(kw, cbh + (size_t)tid * D);
-                ip = tid;
-            }
-            warp_argmin(dp, ip);
-            if (lane == 0) { sD[warp] = dp; sI[warp] = ip; }
-            __syncthreads();
-            dp = lane < 4 ? sD[lane] : INFINITY;
-            ip = lane < 4 ? sI[lane] : p.M0;
-            warp_argmin(dp, ip);
-            bp = ip < p.M0 ? ip : 0;   // (ip == M0 only for non-finite inputs)
-        }
-        if (warp == 0) {
-            // lanes 0..C-1: the children; lane C: the parent
-            double d = INFINITY;
-            if (lane <= C) d = exact_dist_rows<D>(kw, cbh + (size_t)(lane < C ? p.M0 + bp * C + lane : bp) * D);
-            const double dpar = __shfl_sync(0xffffffffu, d, C);
-            int cc = lane < C ? lane : C;
-            if (lane >= C) d = INFINITY;
-            warp_argmin(d, cc);
-            const int leaf = d < dpar ? p.M0 + bp * C + cc : bp;
-            const int old = p.assign[key];
-            if (old != leaf) {
-                const size_t base = (size_t)bh * p.Mtot;
-                if (lane == 0) {
-                    p.assign[key] = leaf;
-                    atomicSub(p.counts + base + old, 1);
-                    atomicAdd(p.counts + base + leaf, 1);
-                }
-                for (int j = lane; j < D; j += 32) {
-                    const float v = __uint_as_float((uint32_t)__ldg(V + key * D + j) << 16);
-                    atomicAdd(p.vsum + (base + old) * D + j, -v);
-                    atomicAdd(p.vsum + (base + leaf) * D + j, v);
-                }
-            }
-        }
-        __syncthreads();   // sD/sI are rewritten for the next key
     }
 }
 
@@ -645,7 +642,7 @@ size_t pre_smem_bytes(int D, int M0, int C, int Mtot) {
     const size_t M0p = (size_t)((M0 + 15) & ~15);
     return 1024 + nwg * (size_t)(D / 64) * kRegion + (size_t)(D / 64) * M0p * 128 +
            (((size_t)M0 * C * D * 2 + 15) & ~size_t(15)) + 128 * 4 /*sCn*/ + 16 * 4 /*sRed*/ +
-           (size_t)M0 * C * 4 /*sCcn*/ + (size_t)Mtot * 4 +
+           (size_t)M0 * C * 4 /*sCcn*/ + (size_t)Mtot * 4 + 4 /*sFix*/ +
            8 + (2 * nwg + 1) * 8 + 16;
 }
 
@@ -676,7 +673,6 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     prm.vsum = vsum;
     prm.status = status;
     // the workspace holds the status block, then the list of open keys
-    prm.fix_count = &status->pad[2];
     prm.fix_list = reinterpret_cast<long long*>(reinterpret_cast<uint8_t*>(status) + kStatusBytes);
     const size_t smem = pre_smem_bytes(D, s.M0, C, Mtot);
     constexpr int NWG = D == 64 ? 4 : 2;
@@ -688,10 +684,6 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = std::min(prm.total_tiles, sms);
     kern<<<grid, 128 * NWG, smem, st>>>(tk, tcb, prm);
-    count_launch();
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    precompute_fixup_kernel<D, C><<<sms * 16, 128, 0, st>>>(prm, static_cast<const uint16_t*>(V));
     count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -78,9 +78,9 @@ typedef enum {
 /*
  * Workspace needed by avq_precompute for `s` (bytes, a multiple of 256;
  * 0 for invalid shapes): 256 bytes for the device status word read by
- * avq_device_status, then 8 bytes per key (B*H*N) for the list of keys whose
- * nearest parent or leaf the kernel's fp32 error bounds leave open; those keys
- * are decided exactly (fp64) by a second pass of the same call.
+ * avq_device_status, then 8 bytes per key (B*H*ceil(N/128)*128) for the list
+ * of keys whose nearest parent or leaf the kernel's fp32 error bounds leave
+ * open; those keys are then decided exactly (fp64) within the same call.
  */
 size_t avq_precompute_workspace_bytes(const avq_shape* s);
 
