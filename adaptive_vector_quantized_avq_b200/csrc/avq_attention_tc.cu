@@ -467,7 +467,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         float2 tt = ffma2(make_float2(sc[j], sc[j + 1]), sl2v, negm);
                         tt = fadd2(tt, e ? make_float2(lc.z, lc.w) : make_float2(lc.x, lc.y));
                         xmax = fmax3(xmax, tt.x, tt.y);
-                        const float2 ev = make_float2(ex2(fminf(tt.x, 126.f)), ex2(fminf(tt.y, 126.f)));
+                        // (past the range bound the weight may overflow: the call reports
+                        // AVQ_ERANGE, and the output is not meaningful)
+                        const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));
                         const float2 wc = ffma2(make_float2(nap[c][j / C], nap[c][(j + 1) / C]),
                                                 e ? make_float2(nc.z, nc.w) : make_float2(nc.x, nc.y), ev);
                         if (e) den1 = fadd2(den1, wc);

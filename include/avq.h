@@ -72,7 +72,7 @@ typedef enum {
                                non-empty child's scaled logit plus log n_c exceeded the common
                                shift of that query's weights (the largest non-empty parent logit
                                plus log n_p) by more than 60 (natural-log units): its weights may
-                               overflow fp32 */
+                               overflow fp32, and O is then not meaningful */
 } avq_status;
 
 /*

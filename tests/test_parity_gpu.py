@@ -84,3 +84,59 @@ def test_full_size_parity(lib_built, oracle, name):
     wl = syn.WORKLOADS[name]
     rep = _run_case(wl, wl.P, oracle, tile_ids_fn=_sample_tiles)
     print(name, rep)
+
+
+def test_duplicate_parents_exact_ties(lib_built, oracle):
+    """Parents 0 and 1 (and their children) are the same codewords, so every
+    key of that cluster is an exact parent tie that no fp32 bound separates:
+    the keys go through the exact fp64 decision, which must keep the lower
+    index (paper §4.2 argmin; ties to the lowest index)."""
+    wl = syn.small_workload(B=1, H=2, N=900, d=64, M0=16, C=4, tile=128, dtype="bf16", seed=11,
+                            n_components=16)
+    inp = syn.generate(wl)
+    cb = inp.codebook.copy()
+    for h in range(wl.H):
+        cb[h, 1] = cb[h, 0]
+        cb[h, wl.M0 + wl.C:wl.M0 + 2 * wl.C] = cb[h, wl.M0:wl.M0 + wl.C]
+    inp = syn.Inputs(wl, inp.K, inp.V, inp.Q, cb)
+    gpu = parity.run_gpu(wl, inp, (0, 4))
+    ora = oracle.precompute(inp.f64("K"), inp.f64("V"), inp.f64("codebook"), wl.M0, wl.C)
+    rep = parity.check_precompute(wl, inp, gpu, ora, oracle)
+    # every key of the duplicated cluster was re-decided, and none landed on parent 1's subtree
+    assert gpu["redecided"][0] > 0
+    sub1 = (gpu["assign"] == 1) | ((gpu["assign"] >= wl.M0 + wl.C) & (gpu["assign"] < wl.M0 + 2 * wl.C))
+    assert not sub1.any()
+    for P in (0, 4):
+        O, sel = gpu["att"][P]
+        parity.check_attention(wl, inp, P, O, sel, ora["counts"], ora["vsum"], oracle)
+    print(rep)
+
+
+def test_range_flag(lib_built):
+    """A non-empty child whose logit lies far above every parent logit of the
+    queries raises AVQ_ERANGE in the attention call's device status (no fault;
+    the tensor-core kernel reports it after the launch)."""
+    from adaptive_vector_quantized_avq_b200 import binding as bd
+    d, M0, C, N = 64, 16, 2, 256
+    rng = np.random.default_rng(12)
+    grid = 1.0 / 32
+    par = np.round(rng.standard_normal((M0, d)) * 0.1 / grid) * grid   # parents near 0 ...
+    par[0] = 0.25                                                       # ... parent 0 a little out
+    ch = np.repeat(par, C, axis=0).copy()
+    ch[0] = 3.0                                                         # child 0 of parent 0: far out
+    cb = np.concatenate([par, ch])[None]                                # [1, Mtot, d]
+    K = np.round(rng.standard_normal((1, 1, N, d)) * 0.1 / grid) * grid
+    K[0, 0, 0] = 3.0                                                    # a key on the far child
+    # q . child0 = 96 against q . parent0 = 8 (scale 1): ~80 nats above the shift
+    Q = np.full((1, 1, N, d), 0.5)
+    dev = "cuda"
+    t = lambda a: parity.to_device(syn.f64_to_bf16_bits(a), "bf16", dev)
+    Kt, Qt, cbt = t(K), t(Q), t(cb)
+    assign, counts, vsum = bd.precompute(Kt, Kt, cbt, M0, C)
+    torch.cuda.synchronize()
+    assert int(assign[0, 0, 0]) == M0   # the far key sits on child 0 of parent 0
+    shape = bd.make_shape(1, 1, N, d, M0, C, Qt.dtype)
+    ws = bd.workspace(bd.avq_attention_workspace_bytes(shape, M0, 128), Qt.device)
+    bd.attention(Qt, cbt, counts, vsum, M0, C, M0, 128, 1.0, ws=ws)
+    assert bd.avq_device_status(ws) == -6
+    assert bd.avq_device_status(ws) == 0   # reading the status clears it
