@@ -1,9 +1,10 @@
 // avq_attention_tc.cu -- tensor-core (tcgen05) kernel of avq_attention for
 // bf16 inputs, 128-query tiles (paper §4.3; papernotes, Key Designs 3).
 //
-// Persistent: CTAs of 128 threads walk contiguous ranges of query tiles
-// (head-major, so a head's parent tables are loaded once per head). Thread r
-// owns query row r of the tile and TMEM lane r.
+// Persistent: CTAs of 256 threads walk contiguous ranges of query tiles
+// (head-major, so a head's parent tables are loaded once per head). Threads r
+// and r + 128 share query row r of the tile (TMEM lane r), each with half of
+// the parent columns, child slots and output dimensions.
 //
 // Weights are kept in log-count form: for parent p the row works with
 // x_p = scale*log2(e)*S_p + log2(n_p) (log2 0 = -inf), so that
@@ -11,7 +12,8 @@
 // contraction then uses per-codeword MEANS (vsum / n), so its weights are the
 // count-weighted e'_p. Per tile:
 //   1. TMA brings the Q tile (prefetched one tile ahead, two stages).
-//   2. MMA1  S_p = Q C_par^T (M=128, N=M0p, K=d) -> TMEM.
+//   2. MMA1  S_p = Q C_par^T (M=128, N=M0p, K=d) -> TMEM (for the next tile
+//      of the same (b,h), issued at the end of the current one).
 //   3. parent pass: x_p, m, e'_p, Zbar = sum e'_p (fp32); bf16(e'_p) -> TMEM
 //      (A operand of MMA3); fp32 e'_p -> TMEM; importance terms e'_p / Zbar
 //      summed over the tile's rows by a warp butterfly + 4-way smem sum.
@@ -19,12 +21,13 @@
 //   5. MMA3p  Xbar = W_par x mean_par issued at once (overlaps the gather).
 //   6. per chunk of <= 128 selected children: gather codewords and means
 //      (cp.async into swizzled smem), MMA2 S_c = Q C_child^T, child weight
-//      (A_c - A_p) n_c (the parent-contribution replacement of the paper's
-//      DeltaA, in count-weighted form), fp32 denominator correction,
-//      bf16 weights -> TMEM, MMA3c accumulates into Xbar.
+//      (A_c - A_p) n_c = 2^(x_c - m + log2 n_c) - A_p n_c (the parent-
+//      contribution replacement of the paper's DeltaA, in count-weighted
+//      form), fp32 denominator correction, bf16 weights -> TMEM, MMA3c
+//      accumulates into Xbar.
 //   7. O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store.
 // Layouts: d = 64 with P*C <= 128 uses 256 TMEM columns (S_c aliases S_p,
-// W_c aliases W_p) and ~101 KB of shared memory, so two CTAs share an SM;
+// W_c aliases W_p) and ~105 KB of shared memory, so two CTAs share an SM;
 // otherwise 512 columns and one CTA per SM.
 #include <algorithm>
 

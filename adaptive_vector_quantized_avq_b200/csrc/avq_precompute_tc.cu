@@ -20,18 +20,20 @@
 //      warpgroup's TMEM columns.
 //   2. a1: v_p = ||C_p||^2 - 2 S_p (the expanded distance minus ||k||^2) in
 //      fp32: the minimum, then the parents within the error bound of this
-//      expanded form; more than one is re-decided with the exact fp64
-//      distance summed in index order.
+//      expanded form; a single one is certainly the nearest.
 //   3. a2: the kept parent and its C children, v = ||C||^2 - 2 k.C with the
 //      dot product on CUDA cores (bf16 x bf16 mixed-precision fma, no
 //      unpacking) under a tighter bound; a child wins only when strictly
-//      closer (parent first, lowest child index among equals); the band the
-//      bound cannot separate is re-decided in fp64.
+//      closer (parent first, lowest child index among equals).
 //   4. a3: assign written; the key counts at its leaf (shared memory,
 //      warp-aggregated) and its V row (read from global memory, coalesced) is
 //      added to the leaf's value sum with 16-byte fp32 vector reductions.
-// A second kernel then adds each parent's children into the parent's totals,
-// so that a parent holds its whole cluster.
+// A key whose parent or leaf the bounds leave open keeps a provisional leaf
+// and is listed; after its last tile the CTA decides its listed keys with
+// exact fp64 distances summed in index order and moves their contributions
+// where the decision changes. A second kernel then adds each parent's
+// children into the parent's totals, so that a parent holds its whole
+// cluster.
 #include <algorithm>
 
 #include "avq_internal.cuh"
@@ -47,7 +49,7 @@ constexpr uint32_t kRegion = 128 * 128;
 
 struct TcPreParams {
     int BH, H, N, M0, M0p, Mtot, ntiles, total_tiles;
-    const uint16_t* K;          // [BH, N, D] bf16 (exact re-decisions read keys here)
+    const uint16_t* K;          // [BH, N, D] bf16
     const uint16_t* V;          // [BH, N, D] bf16
     const uint16_t* codebook;   // [H, Mtot, D] bf16
     int32_t* assign;            // [BH, N]
