@@ -175,44 +175,68 @@ def bus_id_of(torch, dev: int) -> str | None:
 
 # ------------------------------------------------------- CPU oracle timing
 class OracleSampler:
-    """The fp64 oracle timed on a bounded sample of the workload: the first
-    ``n`` keys of head (0,0) through the precompute and the first ``n`` query
-    rows (whole tiles) through the attention, using that head's full
-    statistics (computed once, untimed, like inputs already resident)."""
+    """The fp64 oracle timed on a bounded sample of the workload: whole (b,h)
+    sequences (keys through the precompute, then every query tile through the
+    attention with that sequence's statistics), as many as fit the time budget;
+    when even one sequence does not fit, the first whole tiles of one. Inputs
+    and the statistics the attention reads are prepared untimed, like inputs
+    already resident."""
 
     def __init__(self, wl: syn.Workload, P: int):
         from oracle import oracle as orc
         self.O = orc.get()
         self.threads = self.O.max_threads()
         self.wl, self.P = wl, P
-        one = wl.with_(B=1, H=1)
-        inp = syn.generate(one)
-        self.K, self.V, self.Q, self.cb = (inp.f64(n) for n in ("K", "V", "Q", "codebook"))
-        self.full = self.O.precompute(self.K, self.V, self.cb, wl.M0, wl.C, nthreads=self.threads)
-        self.ntiles = one.ntiles
+        self.one = wl.with_(B=1, H=1)
+        self.ntiles = self.one.ntiles
+        self.heads = [self._head(0)]
+        self.n_heads, self.n_tiles = 1, self.ntiles
 
-    def run(self, n_tiles: int):
+    def _head(self, i: int):
+        inp = syn.generate(self.one.with_(seed=self.wl.seed + 7919 * i))
+        K, V, Q, cb = (inp.f64(n) for n in ("K", "V", "Q", "codebook"))
+        full = self.O.precompute(K, V, cb, self.wl.M0, self.wl.C, nthreads=self.threads)
+        return K, V, Q, cb, full
+
+    def _one(self, h, n_tiles: int) -> int:
         wl = self.wl
-        n_tiles = max(1, min(self.ntiles, n_tiles))
+        K, V, Q, cb, full = h
         n = min(wl.N, n_tiles * wl.tile)
+        self.O.precompute(K[:, :, :n], V[:, :, :n], cb, wl.M0, wl.C, nthreads=self.threads)
+        self.O.attention(Q, cb, full["counts"], full["vsum"], wl.M0, wl.C, self.P, wl.tile,
+                         wl.softmax_scale, tile_ids=np.arange(n_tiles), nthreads=self.threads)
+        return n
+
+    def plan(self, seconds: float) -> None:
+        """Choose the sample for a budget of about `seconds` of oracle work."""
         t0 = time.perf_counter()
-        self.O.precompute(self.K[:, :, :n], self.V[:, :, :n], self.cb, wl.M0, wl.C,
-                          nthreads=self.threads)
-        self.O.attention(self.Q, self.cb, self.full["counts"], self.full["vsum"], wl.M0, wl.C,
-                         self.P, wl.tile, wl.softmax_scale, tile_ids=np.arange(n_tiles),
-                         nthreads=self.threads)
-        return n, time.perf_counter() - t0
+        self._one(self.heads[0], 2)
+        per_row = (time.perf_counter() - t0) / min(self.wl.N, 2 * self.wl.tile)
+        per_head = per_row * self.wl.N
+        if per_head > seconds:
+            self.n_heads = 1
+            self.n_tiles = int(max(1, min(self.ntiles, math.ceil(seconds / per_row / self.wl.tile))))
+        else:
+            self.n_heads = int(max(1, min(self.wl.B * self.wl.H, seconds // per_head)))
+            self.n_tiles = self.ntiles
+            while len(self.heads) < self.n_heads:
+                self.heads.append(self._head(len(self.heads)))
 
-    def tiles_for(self, seconds: float) -> int:
-        n, dt = self.run(2)
-        per_row = dt / n
-        return int(max(1, min(self.ntiles, math.ceil(seconds / per_row / self.wl.tile))))
+    def run(self):
+        t0 = time.perf_counter()
+        rows = sum(self._one(h, self.n_tiles) for h in self.heads[:self.n_heads])
+        return rows, time.perf_counter() - t0
 
-    def describe(self, n_tiles: int) -> str:
-        n = min(self.wl.N, n_tiles * self.wl.tile)
-        return (f"{n} keys precomputed + {n} queries attended ({n_tiles} tiles of "
-                f"{self.wl.tile}) of head (0,0) of {self.wl.name}; fp64 oracle, "
-                f"{self.threads} OpenMP threads")
+    def describe(self) -> str:
+        wl = self.wl
+        if self.n_heads > 1 or self.n_tiles == self.ntiles:
+            what = (f"{self.n_heads} whole (b,h) sequence(s) of {wl.N} keys and {wl.N} queries "
+                    f"of {wl.name} ({self.n_heads * wl.N} rows)")
+        else:
+            n = min(wl.N, self.n_tiles * wl.tile)
+            what = (f"{n} keys precomputed + {n} queries attended ({self.n_tiles} tiles of {wl.tile}) "
+                    f"of one (b,h) sequence of {wl.name}")
+        return f"{what}; fp64 oracle, {self.threads} OpenMP threads"
 
 
 # --------------------------------------------------------------- our arm
@@ -425,10 +449,10 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         smp = OracleSampler(wl, P)
-        nt = smp.tiles_for(args.cpu_budget)
-        n, secs = smp.run(nt)
+        smp.plan(args.cpu_budget)
+        n, secs = smp.run()
         out["cpu_baseline"] = {"value": n / secs, "unit": UNIT, "cores": smp.threads,
-                               "kind": "oracle", "sample": smp.describe(nt), "seconds": secs}
+                               "kind": "oracle", "sample": smp.describe(), "seconds": secs}
     if rank == 0:
         print(json.dumps(out), flush=True)
 
@@ -442,15 +466,15 @@ def run_reference(args):
     P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
     smp = OracleSampler(wl, P)
     per_step = 150.0 / max(1, args.steps + args.warmup)
-    nt = smp.tiles_for(per_step)          # calibration, untimed
+    smp.plan(per_step)                    # calibration and input preparation, untimed
     for _ in range(args.warmup):
-        smp.run(nt)
+        smp.run()
     times = []
     for _ in range(args.steps):
-        n, dt = smp.run(nt)
+        n, dt = smp.run()
         times.append(dt)
     rows = n
-    cores, desc = smp.threads, smp.describe(nt)
+    cores, desc = smp.threads, smp.describe()
     ms = 1e3 * statistics.mean(times)
     value = rows / (ms / 1e3)
     print(json.dumps({
