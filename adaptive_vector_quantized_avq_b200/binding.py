@@ -26,7 +26,7 @@ _STATUS = {0: "AVQ_OK", -1: "AVQ_EINVAL", -2: "AVQ_EUNSUPPORTED", -3: "AVQ_ECUDA
 # every symbol include/avq.h declares (checked by the tests)
 EXPORTS = ("avq_precompute_workspace_bytes", "avq_precompute", "avq_attention_workspace_bytes",
            "avq_attention", "avq_device_status", "avq_status_string", "avq_version",
-           "avq_kernel_launches", "avq_attention_noalloc")
+           "avq_kernel_launches", "avq_attention_noalloc", "avq_commitment")
 
 
 class AVQError(RuntimeError):
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.avq_attention_noalloc.argtypes = [shp, vp, vp, vp, vp, i32, i32, ctypes.c_float, vp, vp,
                                             vp, vp]
         L.avq_attention_noalloc.restype = i32
+        L.avq_commitment.argtypes = [shp, vp, vp, vp, vp, vp]
+        L.avq_commitment.restype = i32
         L.avq_kernel_launches.argtypes = []
         L.avq_kernel_launches.restype = ctypes.c_uint64
         _LIB = L
@@ -146,6 +148,11 @@ def avq_attention_noalloc(shape, Q, codebook, counts, vsum, P, tile, scale, O, s
     return lib().avq_attention_noalloc(ctypes.byref(shape), _ptr(Q), _ptr(codebook), _ptr(counts),
                                        _ptr(vsum), P, tile, float(scale), _ptr(O), _ptr(selected),
                                        _ptr(device_status), _stream(stream))
+
+
+def avq_commitment(shape, K, codebook, assign, sq_err, stream=None) -> int:
+    return lib().avq_commitment(ctypes.byref(shape), _ptr(K), _ptr(codebook), _ptr(assign), _ptr(sq_err),
+                                _stream(stream))
 
 
 def avq_device_status(workspace, stream=None) -> int:
@@ -219,4 +226,22 @@ def attention(Q: torch.Tensor, codebook: torch.Tensor, counts: torch.Tensor, vsu
                        out[1] if P > 0 else None, ws, ws.numel(), stream)
     if rc != AVQ_OK:
         raise AVQError(rc, "avq_attention")
+    return out
+
+
+def commitment(K: torch.Tensor, codebook: torch.Tensor, assign: torch.Tensor, M0: int, C: int,
+               *, stream=None) -> torch.Tensor:
+    """Per-(b,h) sum of ||k - codebook[h, assign]||^2 over the keys ([B,H] fp64);
+    divide by N for the commitment loss."""
+    _check(K, "K")
+    _check(codebook, "codebook", K.dtype)
+    _check(assign, "assign", torch.int32)
+    B, H, N, d = K.shape
+    if assign.shape != (B, H, N) or codebook.shape != (H, M0 * (1 + C), d):
+        raise ValueError(f"shapes: K {tuple(K.shape)}, assign {tuple(assign.shape)}, codebook "
+                         f"{tuple(codebook.shape)}")
+    out = torch.empty((B, H), dtype=torch.float64, device=K.device)
+    rc = avq_commitment(make_shape(B, H, N, d, M0, C, K.dtype), K, codebook, assign, out, stream)
+    if rc != AVQ_OK:
+        raise AVQError(rc, "avq_commitment")
     return out

@@ -173,6 +173,27 @@ int avq_attention_noalloc(const avq_shape* s, const void* Q, const void* codeboo
                           void* O, int32_t* selected, int32_t* device_status, void* stream);
 
 /*
+ * Commitment loss of an assignment (paper, appendix "Per-layer codebook
+ * analysis", Table 7: the mean squared distance between each key and its
+ * assigned codeword; here the assigned codeword is the key's leaf, as written
+ * to `assign` by avq_precompute). A diagnostic, outside the forward path.
+ *
+ * For every (b,h): sq_err[b*H + h] = sum over n of
+ *   ||K[b,h,n] - codebook[h, assign[b,h,n]]||^2
+ * (divide by N for the mean). Each squared difference is taken in fp32 from
+ * the stored values, the sums are accumulated in fp64 (order unspecified).
+ * A leaf id outside [0, M0*(1+C)) makes its (b,h) sum NaN.
+ *
+ * K, codebook: device, as for avq_precompute (16-byte aligned). assign:
+ * device [B,H,N] int32 (4-byte aligned). sq_err: device, B*H doubles
+ * (8-byte aligned), overwritten. Returns AVQ_OK, AVQ_EINVAL (null or
+ * misaligned pointer, invalid shape), AVQ_EUNSUPPORTED, AVQ_ECUDA. Does not
+ * synchronise.
+ */
+int avq_commitment(const avq_shape* s, const void* K, const void* codebook, const int32_t* assign,
+                   double* sq_err, void* stream);
+
+/*
  * Blocking: waits for `stream`, then reads the status word that kernels of
  * earlier calls using `workspace` left there (AVQ_OK; AVQ_ETIMEOUT when a
  * bounded device-side wait ran out; AVQ_ERANGE, see above) and clears it.

@@ -136,6 +136,22 @@ class Oracle:
         return out
 
 
+def commitment(K: np.ndarray, codebook: np.ndarray, assign: np.ndarray) -> np.ndarray:
+    """Per-(b,h) sum over the keys of ||k - codebook[h, assign]||^2 in fp64
+    (paper, appendix "Per-layer codebook analysis", Table 7: the commitment
+    loss is this sum divided by N; the assigned codeword is the key's leaf).
+    K [B,H,N,d], codebook [H,Mtot,d], assign [B,H,N] -> [B,H]."""
+    K = np.asarray(K, dtype=np.float64)
+    cb = np.asarray(codebook, dtype=np.float64)
+    B, H, N, d = K.shape
+    out = np.zeros((B, H))
+    for b in range(B):
+        for h in range(H):
+            diff = K[b, h] - cb[h][assign[b, h]]
+            out[b, h] = float((diff * diff).sum())
+    return out
+
+
 _DEFAULT: Oracle | None = None
 
 
