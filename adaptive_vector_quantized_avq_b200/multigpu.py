@@ -5,8 +5,16 @@ so the path shards with no data-path collective: each rank runs the whole
 forward pass on its own batch (weak scaling). The only collectives are the
 ones that time the job: a barrier around the timed region and a MAX
 all-reduce of the per-rank times, so that the reported time is the slowest
-rank's. These helpers work with any torch.distributed backend (nccl on the
-GPUs, gloo on the CPU for tests).
+rank's.
+
+For few, long sequences the keys and queries of each (b,h) can instead be
+split along N (``sequence_sharded_forward``): every rank assigns its own keys,
+one SUM all-reduce of the counts and value sums makes the statistics global,
+and every rank attends its own queries. Selection depends only on the global
+statistics and on tiles, so tiles must not straddle ranks.
+
+These helpers work with any torch.distributed backend (nccl on the GPUs, gloo
+on the CPU for tests).
 """
 from __future__ import annotations
 
@@ -58,3 +66,35 @@ def max_over_ranks(values, device: torch.device | None = None) -> list[float]:
 def weak_scaling_value(rows_per_rank: int, world: int, ms_per_step: float) -> float:
     """Whole-job throughput: all ranks' query rows per second of the slowest rank."""
     return rows_per_rank * world / (ms_per_step / 1e3)
+
+
+def shard_rows(N: int, world: int, rank: int, tile: int) -> tuple[int, int]:
+    """Rows [n0, n1) of a length-N sequence held by `rank` when the sequence is
+    split along N into `world` runs of whole tiles (the last rank takes the
+    ragged end)."""
+    ntiles = (N + tile - 1) // tile
+    t0, t1 = (ntiles * rank) // world, (ntiles * (rank + 1)) // world
+    return min(N, t0 * tile), min(N, t1 * tile)
+
+
+def sequence_sharded_forward(K, V, Q, codebook, M0: int, C: int, P: int, tile: int, scale: float,
+                             *, precompute=None, attention=None, group=None):
+    """The forward path with the keys and queries of every (b,h) split along N
+    across the ranks of `group` (``shard_rows`` gives each rank's rows; every
+    local N but the last must be a whole number of tiles, so that local tiles
+    are global tiles). K, V, Q: this rank's [B,H,n,d]; codebook: the full
+    [H,Mtot,d]. Returns (assign of the local keys, global counts, global vsum,
+    O of the local queries, selected of the local tiles).
+
+    `precompute` / `attention` default to the library calls of ``binding``
+    (callables with their signatures may be passed instead, e.g. by tests)."""
+    if precompute is None or attention is None:
+        from . import binding
+        precompute = precompute or binding.precompute
+        attention = attention or binding.attention
+    assign, counts, vsum = precompute(K, V, codebook, M0, C)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(counts, op=dist.ReduceOp.SUM, group=group)
+        dist.all_reduce(vsum, op=dist.ReduceOp.SUM, group=group)
+    O, selected = attention(Q, codebook, counts, vsum, M0, C, P, tile, scale)
+    return assign, counts, vsum, O, selected
