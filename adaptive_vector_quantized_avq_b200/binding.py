@@ -26,7 +26,8 @@ _STATUS = {0: "AVQ_OK", -1: "AVQ_EINVAL", -2: "AVQ_EUNSUPPORTED", -3: "AVQ_ECUDA
 # every symbol include/avq.h declares (checked by the tests)
 EXPORTS = ("avq_precompute_workspace_bytes", "avq_precompute", "avq_attention_workspace_bytes",
            "avq_attention", "avq_device_status", "avq_status_string", "avq_version",
-           "avq_kernel_launches", "avq_attention_noalloc", "avq_commitment")
+           "avq_kernel_launches", "avq_attention_noalloc", "avq_commitment", "avq_gilbert_order",
+           "avq_gather_rows")
 
 
 class AVQError(RuntimeError):
@@ -79,6 +80,10 @@ def lib() -> ctypes.CDLL:
         L.avq_attention_noalloc.restype = i32
         L.avq_commitment.argtypes = [shp, vp, vp, vp, vp, vp]
         L.avq_commitment.restype = i32
+        L.avq_gilbert_order.argtypes = [i32, i32, vp]
+        L.avq_gilbert_order.restype = i32
+        L.avq_gather_rows.argtypes = [shp, vp, vp, vp, vp]
+        L.avq_gather_rows.restype = i32
         L.avq_kernel_launches.argtypes = []
         L.avq_kernel_launches.restype = ctypes.c_uint64
         _LIB = L
@@ -153,6 +158,15 @@ def avq_attention_noalloc(shape, Q, codebook, counts, vsum, P, tile, scale, O, s
 def avq_commitment(shape, K, codebook, assign, sq_err, stream=None) -> int:
     return lib().avq_commitment(ctypes.byref(shape), _ptr(K), _ptr(codebook), _ptr(assign), _ptr(sq_err),
                                 _stream(stream))
+
+
+def avq_gilbert_order(rows: int, cols: int, order) -> int:
+    """`order`: a writable host buffer of rows*cols int32 (e.g. a numpy array)."""
+    return lib().avq_gilbert_order(rows, cols, order.ctypes.data if hasattr(order, "ctypes") else order)
+
+
+def avq_gather_rows(shape, src, dst, perm, stream=None) -> int:
+    return lib().avq_gather_rows(ctypes.byref(shape), _ptr(src), _ptr(dst), _ptr(perm), _stream(stream))
 
 
 def avq_device_status(workspace, stream=None) -> int:
@@ -245,3 +259,28 @@ def commitment(K: torch.Tensor, codebook: torch.Tensor, assign: torch.Tensor, M0
     if rc != AVQ_OK:
         raise AVQError(rc, "avq_commitment")
     return out
+
+
+def gilbert_order(rows: int, cols: int):
+    """The tokens of a rows x cols grid (token r*cols + c) in Gilbert-curve
+    order, as an int32 numpy array (host)."""
+    import numpy as np
+    order = np.empty(rows * cols, dtype=np.int32)
+    rc = avq_gilbert_order(rows, cols, order)
+    if rc != AVQ_OK:
+        raise AVQError(rc, "avq_gilbert_order")
+    return order
+
+
+def gather_rows(x: torch.Tensor, perm: torch.Tensor, *, stream=None) -> torch.Tensor:
+    """y[b,h,i,:] = x[b,h,perm[i],:] for a [B,H,N,d] tensor (device kernel)."""
+    _check(x, "x")
+    _check(perm, "perm", torch.int32)
+    B, H, N, d = x.shape
+    if perm.shape != (N,):
+        raise ValueError(f"perm must have shape ({N},), got {tuple(perm.shape)}")
+    y = torch.empty_like(x)
+    rc = avq_gather_rows(make_shape(B, H, N, d, 1, 1, x.dtype), x, y, perm, stream)
+    if rc != AVQ_OK:
+        raise AVQError(rc, "avq_gather_rows")
+    return y

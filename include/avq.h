@@ -194,6 +194,32 @@ int avq_commitment(const avq_shape* s, const void* K, const void* codebook, cons
                    double* sq_err, void* stream);
 
 /*
+ * Query reordering along a Gilbert space-filling curve (paper §4.2,
+ * "Per-query-tile amortization and adaptivity"; appendix "Spatial reordering
+ * ablation", Table 8): tokens laid out on a rows x cols grid (token
+ * t = r*cols + c) are reordered so that consecutive tokens are grid
+ * neighbours and every run of T consecutive tokens (a query tile) covers a
+ * compact 2-D region, for any grid size (the Gilbert curve generalises the
+ * Hilbert curve to rectangles).
+ *
+ * avq_gilbert_order (host): order[i] = the token visited i-th, a permutation
+ * of 0 .. rows*cols-1. order: host array of rows*cols int32, written.
+ * Returns AVQ_OK or AVQ_EINVAL (rows or cols < 1, rows*cols >= 2^31, null).
+ */
+int avq_gilbert_order(int rows, int cols, int32_t* order);
+
+/*
+ * Row gather along the sequence (device): dst[b,h,i,:] = src[b,h,perm[i],:]
+ * for i < s->N, with the row size of `s` (d elements of s->dtype). With
+ * perm = a Gilbert order this reorders Q (or K, V) before the calls; with its
+ * inverse it restores O afterwards. src, dst: device [B,H,N,d] (16-byte
+ * aligned, not overlapping); perm: device, N int32, each in [0, N) (rows
+ * outside are not read: dst row i is then zeroed). Returns AVQ_OK,
+ * AVQ_EINVAL, AVQ_ECUDA. Does not synchronise.
+ */
+int avq_gather_rows(const avq_shape* s, const void* src, void* dst, const int32_t* perm, void* stream);
+
+/*
  * Blocking: waits for `stream`, then reads the status word that kernels of
  * earlier calls using `workspace` left there (AVQ_OK; AVQ_ETIMEOUT when a
  * bounded device-side wait ran out; AVQ_ERANGE, see above) and clears it.
