@@ -142,6 +142,19 @@ __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* v) {
     tmem_touch16f(v + 16);
 }
 
+// The number of keys among k32[c0 .. c0+63] larger than parent r's in the
+// order (key, complement of the index): ties go to the lower index. Not
+// inlined: it runs only for tiles whose leading ranks tie.
+__device__ __noinline__ int count_larger_keys64(const uint32_t* k32, int c0, uint32_t kr, int r) {
+    const unsigned long long key = ((unsigned long long)kr << 32) | (uint32_t)(0xFFFFFFFFu - r);
+    int rk = 0;
+    for (int q = 0; q < 64; ++q) {
+        const unsigned long long kq = ((unsigned long long)k32[c0 + q] << 32) | (uint32_t)(0xFFFFFFFFu - (c0 + q));
+        rk += kq > key;
+    }
+    return rk;
+}
+
 // pair barrier: the two warps (w and w+4) that share TMEM lanes 32w..32w+31
 __device__ __forceinline__ void pair_sync(int quarter) {
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
@@ -346,34 +359,50 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         if (__syncthreads_or(!ok)) { failed = true; break; }
 
-        // ---- importance and top-P selection: ranks over 64-bit keys, each
-        // thread of a pair counting over half of the parents
+        // ---- importance and top-P selection. The key of a parent is the bit
+        // pattern of its importance (w >= 0 orders like its bits; padding
+        // parents 0); its rank is the number of larger keys, ties to the lower
+        // index. Each thread of a pair counts the strictly larger keys among
+        // half of the parents with 32-bit compares; when the P leading ranks
+        // are free of ties (every candidate lands on its own slot) those are
+        // the ranks. Otherwise the tile is ranked again over 64-bit keys
+        // (importance bits, then the complement of the index).
         {
+            uint32_t* sK32 = reinterpret_cast<uint32_t*>(sKey);
             if (tid < 128) {
                 const float w = (sPart[tid] + sPart[128 + tid]) + (sPart[256 + tid] + sPart[384 + tid]);
-                // larger importance first, then the lower index; w >= 0 orders like its bits
-                sKey[tid] = tid < p.M0 ? ((unsigned long long)__float_as_uint(w) << 32) |
-                                             (uint32_t)(0xFFFFFFFFu - tid)
-                                       : 0ull;
+                sK32[tid] = tid < p.M0 ? __float_as_uint(w) : 0u;
             }
             __syncthreads();
-            const unsigned long long key = sKey[r];
-            int rk = 0;
-#pragma unroll 8
-            for (int q = 0; q < 64; q += 2) {
-                const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(sKey + c0 + q);
-                rk += (kk.x > key) + (kk.y > key);
+            const uint32_t kr = sK32[r];
+            int gt = 0;
+#pragma unroll 4
+            for (int q = 0; q < 64; q += 4) {
+                const uint4 kk = *reinterpret_cast<const uint4*>(sK32 + c0 + q);
+                gt += (kk.x > kr) + (kk.y > kr) + (kk.z > kr) + (kk.w > kr);
             }
-            sRank[hf * 128 + r] = rk;
-            pair_sync(quarter);   // the pair's two partial ranks
+            sRank[hf * 128 + r] = gt;
+            pair_sync(quarter);   // the pair's two partial counts
+            int rank = -1;
             if (tid < p.M0) {
-                const int rank = sRank[tid] + sRank[128 + tid];
-                if (rank < p.P) {
-                    sSel[rank] = tid;
-                    p.selected[((size_t)bh * p.ntiles + t) * p.P + rank] = tid;
+                rank = sRank[tid] + sRank[128 + tid];
+                if (rank < p.P) sSel[rank] = tid;
+            }
+            // a candidate that does not find itself in its slot shares its key
+            const bool tie = __syncthreads_or(rank >= 0 && rank < p.P && sSel[rank] != tid);
+            if (tie) {
+                const int rk = count_larger_keys64(sK32, c0, kr, r);
+                __syncthreads();   // every thread has read the slots it checked
+                sRank[hf * 128 + r] = rk;
+                pair_sync(quarter);
+                rank = -1;
+                if (tid < p.M0) {
+                    rank = sRank[tid] + sRank[128 + tid];
+                    if (rank < p.P) sSel[rank] = tid;
                 }
             }
-            __syncthreads();
+            if (rank >= 0 && rank < p.P) p.selected[((size_t)bh * p.ntiles + t) * p.P + rank] = tid;
+            if (tie) __syncthreads();
         }
 
         // ---- parents' value contribution (overlaps the child gather)
