@@ -28,6 +28,14 @@ cudaError_t launch_precompute_tc(const avq_shape& s, const void* K, const void* 
                                  int32_t* assign, int32_t* counts, float* vsum, StatusBlock* status,
                                  cudaStream_t st);
 size_t attention_tc_workspace(const avq_shape& s);
+bool flat_precompute_supported(const avq_shape& s);
+cudaError_t launch_flat_precompute(const avq_shape& s, const void* K, const void* V, const void* cb,
+                                   int32_t* assign, int32_t* counts, float* vsum, StatusBlock* status,
+                                   cudaStream_t st);
+bool flat_attention_supported(const avq_shape& s, int P, int tile);
+cudaError_t launch_flat_attention(const avq_shape& s, const void* Q, const void* cb, const int32_t* counts,
+                                  const float* vsum, float scale, void* O, void* means, StatusBlock* status,
+                                  cudaStream_t st);
 cudaError_t launch_attention_tc(const avq_shape& s, const void* Q, const void* cb, const int32_t* counts,
                                 const float* vsum, int P, float scale, void* O, int32_t* selected,
                                 void* vtab, StatusBlock* status, cudaStream_t st);
@@ -44,8 +52,9 @@ int check_shape(const avq_shape* s) {
     if (s->B < 1 || s->H < 1 || s->N < 0) return AVQ_EINVAL;
     if (s->d != 64 && s->d != 128) return AVQ_EINVAL;
     if (s->dtype != AVQ_F32 && s->dtype != AVQ_BF16) return AVQ_EINVAL;
-    if (s->M0 < 1 || s->C < 1) return AVQ_EINVAL;
-    if (s->M0 > kMaxM0 || s->C > kMaxC) return AVQ_EUNSUPPORTED;
+    if (s->M0 < 1 || s->C < 0) return AVQ_EINVAL;
+    // a tree holds up to kMaxM0 parents; a flat codebook (C == 0) up to kMaxFlat codewords
+    if (s->M0 > (s->C == 0 ? kMaxFlat : kMaxM0) || s->C > kMaxC) return AVQ_EUNSUPPORTED;
     // element counts must fit the kernels' index arithmetic
     const long long rows = (long long)s->B * s->H * s->N;
     if (rows * s->d >= (1LL << 40)) return AVQ_EUNSUPPORTED;
@@ -116,7 +125,8 @@ int avq_precompute(const avq_shape* s, const void* K, const void* V, const void*
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t Mtot = (size_t)s->M0 * (1 + s->C);
     const size_t BH = (size_t)s->B * s->H;
-    const bool tc = s->N > 0 && precompute_tc_supported(*s);
+    if (s->C == 0 && !flat_precompute_supported(*s)) return AVQ_EUNSUPPORTED;
+    const bool tc = s->N > 0 && s->C > 0 && precompute_tc_supported(*s);
     StatusBlock* status = static_cast<StatusBlock*>(workspace);
     {
         // counts and vsum start at zero
@@ -129,7 +139,9 @@ int avq_precompute(const avq_shape* s, const void* K, const void* V, const void*
     }
     if (s->N == 0) return AVQ_OK;
     cudaError_t e;
-    if (tc) {
+    if (s->C == 0) {
+        e = launch_flat_precompute(*s, K, V, codebook, assign, counts, vsum, status, st);
+    } else if (tc) {
         e = launch_precompute_tc(*s, K, V, codebook, assign, counts, vsum, status, st);
     } else {
         e = launch_precompute_simt(*s, K, V, codebook, assign, counts, vsum, st);
@@ -141,7 +153,12 @@ size_t avq_attention_workspace_bytes(const avq_shape* s, int P, int tile) {
     if (check_shape(s) != AVQ_OK) return 0;
     if (P < 0 || P > s->M0 || (tile != 64 && tile != 128)) return 0;
     size_t n = kStatusBytes;
-    if (attention_tc_supported(*s, tile)) n += attention_tc_workspace(*s);
+    if (s->C == 0) {
+        if (!flat_attention_supported(*s, P, tile)) return 0;
+        n += attention_tc_workspace(*s);
+    } else if (attention_tc_supported(*s, tile)) {
+        n += attention_tc_workspace(*s);
+    }
     return n;
 }
 
@@ -151,6 +168,8 @@ int avq_attention(const avq_shape* s, const void* Q, const void* codebook, const
     int rc = check_shape(s);
     if (rc != AVQ_OK) return rc;
     if (P < 0 || P > s->M0 || (tile != 64 && tile != 128)) return AVQ_EINVAL;
+    if (s->C == 0 && P != 0) return AVQ_EINVAL;   // a flat codebook has nothing to select
+    if (s->C == 0 && !flat_attention_supported(*s, P, tile)) return AVQ_EUNSUPPORTED;
     if (!(scale > 0.f) || !(scale < 3.0e38f)) return AVQ_EINVAL;
     if (!codebook || !counts || !vsum) return AVQ_EINVAL;
     if (s->N > 0 && (!Q || !O || (P > 0 && !selected))) return AVQ_EINVAL;
@@ -162,7 +181,11 @@ int avq_attention(const avq_shape* s, const void* Q, const void* codebook, const
     if (s->N == 0) return AVQ_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (attention_tc_supported(*s, tile)) {
+    if (s->C == 0) {
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        e = launch_flat_attention(*s, Q, codebook, counts, vsum, scale, O, ws + kStatusBytes,
+                                  reinterpret_cast<StatusBlock*>(ws), st);
+    } else if (attention_tc_supported(*s, tile)) {
         uint8_t* ws = static_cast<uint8_t*>(workspace);
         e = launch_attention_tc(*s, Q, codebook, counts, vsum, P, scale, O, selected, ws + kStatusBytes,
                                 reinterpret_cast<StatusBlock*>(ws), st);

@@ -584,6 +584,229 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
 }
 
+// Flat codebook (no children, nothing selected) with up to 512 codewords:
+// VQ attention over all of them (paper §3.2, Eq. 3: softmax weights with a
+// log-count bias, per-codeword value means). The codewords' logits come
+// through TMEM in chunks of at most 128, twice per tile: first for the row
+// maximum m of x_p = scale*log2(e)*S_p + log2 n_p, then for e'_p = 2^(x_p - m),
+// Zbar = sum e'_p and the value contraction Xbar += W_chunk x mean_chunk
+// (MMA3, accumulated in TMEM across the chunks). One CTA of 256 threads per
+// SM; threads r and r + 128 share query row r, each with half of every chunk.
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+flat_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                      const __grid_constant__ CUtensorMap tmCB, const __grid_constant__ CUtensorMap tmMN,
+                      const TcAttnParams p) {
+    constexpr int KH = D / 64;
+    constexpr uint32_t IMG = KH * kRegion;
+    constexpr int KSTEPS = D / 16;
+    constexpr int OD = D / 2;
+    constexpr uint32_t colW = 128, colO = 192;               // TMEM: S 0..127, W 128..191, O 192..
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = align1024(smem_raw);
+    const int M0c = (p.M0 + 127) & ~127;
+    const int nchunks = M0c / 128;
+    uint8_t* const sQ0 = base;                                // two Q stages
+    uint8_t* sStage = base + 2 * IMG;                         // O staging
+    uint8_t* sB1 = base + 3 * IMG;                            // codewords (K-major), M0c rows
+    uint8_t* sMn = sB1 + (size_t)KH * M0c * 128;              // value means (MN-major), M0c rows
+    float* sLb = reinterpret_cast<float*>(sMn + (size_t)KH * M0c * 128);   // [M0c] log2 n (-inf if empty)
+    float* sX = sLb + M0c;                                    // [2][128] row exchange
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 256);   // q0, q1, mma, head
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = tid & 127, hf = tid >> 7, quarter = warp & 3;
+    const int g0 = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
+    const int g1 = (int)(((long long)(blockIdx.x + 1) * p.total_tiles) / gridDim.x);
+    if (warp == 0) {
+        tmem_alloc(sTmem, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmO);
+        tma_prefetch_desc(&tmCB);
+        tma_prefetch_desc(&tmMN);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sTmem;
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t idesc3 = idesc_bf16_f32(128, D, true);
+    const int M0p = (p.M0 + 15) & ~15;
+    uint32_t qph = 0, mphase = 0, hphase = 0;
+    bool failed = false;
+    int cur_bh = -1;
+
+    auto issue_q = [&](int g, int stage) {
+        const int bh = g / p.ntiles, t = g % p.ntiles;
+        mbar_arrive_expect_tx(&bars[stage], IMG);
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh)
+            tma_load_3d(sQ0 + stage * IMG + kh * kRegion, &tmQ, &bars[stage], kh * 64, t * kTile, bh);
+    };
+    // logits of codeword chunk j (thread 0 issues; every thread waits)
+    auto chunk_logits = [&](int j, int stage, bool& ok) {
+        if (tid == 0 && ok) {
+            const int nj = min(128, M0p - 128 * j);
+            const uint32_t idesc1 = idesc_bf16_f32(128, nj, false);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks)
+                mma_ss(tmem, desc_k(sQ0 + stage * IMG, ks),
+                       smem_desc_sw128(smem_u32(sB1 + j * 16384) + (uint32_t)(ks >> 2) * (uint32_t)M0c * 128u +
+                                           (uint32_t)(ks & 3) * 32u, 16, 1024),
+                       idesc1, ks > 0);
+            mma_commit(&bars[2]);
+        }
+        ok = mbar_wait(&bars[2], mphase) && ok;
+        mphase ^= 1;
+        tc_fence_after();
+    };
+    // this thread's 64 columns of the chunk (as x = scale*log2e*S + log2 n; -inf past the codebook)
+    auto load_x = [&](int j, float* x) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int col = 128 * j + 64 * hf + 16 * b;
+            if (col < M0p) tmem_ld16f(trow + 64 * hf + 16 * b, x + 16 * b);
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            tmem_touch16f(x + 16 * b);
+            const int col = 128 * j + 64 * hf + 16 * b;
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                x[16 * b + k] = col < M0p ? fmaf(x[16 * b + k], p.sl2, sLb[col + k]) : -INFINITY;
+        }
+    };
+
+    if (tid == 0 && g0 < g1) issue_q(g0, 0);
+    for (int g = g0, it = 0; g < g1; ++g, ++it) {
+        const int stage = it & 1;
+        const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
+        if (tid == 0) bulk_wait_read_all();
+        bool ok = true;
+        if (bh != cur_bh) {   // head change: codewords, means, log-counts
+            __syncthreads();   // every MMA of the previous head has completed (waited by all)
+            if (tid == 0) {
+                mbar_arrive_expect_tx(&bars[3], 2u * KH * (uint32_t)M0c * 128u);
+                for (int kh = 0; kh < KH; ++kh)
+                    for (int r0 = 0; r0 < M0c; r0 += 128) {
+                        tma_load_3d(sB1 + kh * M0c * 128 + r0 * 128, &tmCB, &bars[3], kh * 64, r0, h);
+                        tma_load_3d(sMn + kh * M0c * 128 + r0 * 128, &tmMN, &bars[3], kh * 64, r0, bh);
+                    }
+            }
+            for (int i = tid; i < M0c; i += 256) {
+                const int n = i < p.M0 ? __ldg(p.counts + (size_t)bh * p.Mtot + i) : 0;
+                sLb[i] = n > 0 ? __log2f((float)n) : -INFINITY;
+            }
+            ok = mbar_wait(&bars[3], hphase);
+            hphase ^= 1;
+            if (__syncthreads_or(!ok)) { failed = true; break; }
+            cur_bh = bh;
+        }
+        if (tid == 0) {
+            ok = mbar_wait(&bars[stage], (qph >> stage) & 1u);
+            qph ^= 1u << stage;
+            if (ok && g + 1 < g1) issue_q(g + 1, stage ^ 1);
+        }
+        // pass 1: the row maximum
+        float mx = -INFINITY;
+        for (int j = 0; j < nchunks; ++j) {
+            chunk_logits(j, stage, ok);
+            float x[64];
+            load_x(j, x);
+#pragma unroll
+            for (int k = 0; k < 64; k += 2) mx = fmax3(mx, x[k], x[k + 1]);
+            tc_fence_before();
+            __syncthreads();   // S is free for the next chunk
+        }
+        sX[hf * 128 + r] = mx;
+        pair_sync(quarter);
+        const float m = fmaxf(sX[r], sX[128 + r]);
+        pair_sync(quarter);
+        // pass 2: weights, Zbar and the value contraction
+        float2 zp = make_float2(0.f, 0.f);
+        for (int j = 0; j < nchunks; ++j) {
+            chunk_logits(j, stage, ok);   // (its wait also covers the previous chunk's MMA3)
+            float x[64];
+            load_x(j, x);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                uint32_t w[8];
+#pragma unroll
+                for (int k = 0; k < 16; k += 2) {
+                    const float e0 = ex2(x[16 * b + k] - m), e1 = ex2(x[16 * b + k + 1] - m);
+                    zp = fadd2(zp, make_float2(e0, e1));
+                    w[k >> 1] = pack_bf16x2(e0, e1);
+                }
+                tmem_st8(trow + colW + 32 * hf + 8 * b, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            if (__syncthreads_or(!ok)) { failed = true; break; }
+            if (tid == 0) {
+                const int nj = min(128, M0p - 128 * j);
+                tc_fence_after();
+                for (int ks = 0; ks < nj / 16; ++ks)
+                    mma_ts(tmem + colO, tmem + colW + 8 * ks,
+                           smem_desc_sw128(smem_u32(sMn + j * 16384) + (uint32_t)ks * 2048u, (uint32_t)M0c * 128u, 1024),
+                           idesc3, j > 0 || ks > 0);
+                if (j + 1 == nchunks) mma_commit(&bars[2]);
+            }
+        }
+        if (failed) break;
+        ok = mbar_wait(&bars[2], mphase) && ok;   // the last MMA3
+        mphase ^= 1;
+        tc_fence_after();
+        // epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
+        sX[hf * 128 + r] = zp.x + zp.y;
+        pair_sync(quarter);
+        const float inv = 1.f / (sX[r] + sX[128 + r]);
+        const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+        for (int c = 0; c < OD / 32; ++c) {
+            float o[32];
+            tmem_ld32f(trow + colO + hf * OD + 32 * c, o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t uu[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 v = fmul2(make_float2(o[8 * q + 2 * i], o[8 * q + 2 * i + 1]), inv2);
+                    uu[i] = pack_bf16x2(v.x, v.y);
+                }
+                *reinterpret_cast<uint4*>(sStage + swz(r, hf * (OD / 8) + 4 * c + q)) =
+                    make_uint4(uu[0], uu[1], uu[2], uu[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(!ok)) { failed = true; break; }
+        if (tid == 0) {
+#pragma unroll
+            for (int kh = 0; kh < KH; ++kh) tma_store_3d(&tmO, sStage + kh * kRegion, kh * 64, t * kTile, bh);
+            bulk_commit();
+        }
+    }
+    if (failed && tid == 0) {
+        atomicExch(&p.status->error, (int)AVQ_ETIMEOUT);
+        atomicExch(&p.status->where, (int)blockIdx.x);
+    }
+    if (tid == 0) bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
 // bf16 value means vsum / n (0 for empty codewords): B operand of the value contraction.
 __global__ void means_bf16_kernel(const float4* __restrict__ vsum, const int32_t* __restrict__ counts,
                                   uint2* __restrict__ dst, size_t nrows, int d4) {
@@ -651,6 +874,60 @@ cudaError_t launch_tc(const avq_shape& s, const void* Q, const void* cb, const i
 }
 
 }  // namespace
+
+size_t flat_attn_smem(int D, int M0) {
+    const size_t M0c = (size_t)((M0 + 127) & ~127);
+    return 1024 + 3 * (size_t)(D / 64) * kRegion + 2 * (size_t)(D / 64) * M0c * 128 + M0c * 4 + 256 * 4 + 64;
+}
+
+bool flat_attention_supported(const avq_shape& s, int P, int tile) {
+    return s.dtype == AVQ_BF16 && s.d == 64 && s.C == 0 && P == 0 && tile == kTile && s.M0 <= 512 &&
+           flat_attn_smem(s.d, s.M0) <= 227 * 1024;
+}
+
+cudaError_t launch_flat_attention(const avq_shape& s, const void* Q, const void* cb, const int32_t* counts,
+                                  const float* vsum, float scale, void* O, void* means, StatusBlock* status,
+                                  cudaStream_t st) {
+    constexpr int D = 64;
+    const size_t nrows = (size_t)s.B * s.H * s.M0;
+    means_bf16_kernel<<<(unsigned)std::min<size_t>((nrows * (D / 4) + 255) / 256, 4096), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(vsum), counts, reinterpret_cast<uint2*>(means), nrows, D / 4);
+    count_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int BH = s.B * s.H;
+    CUtensorMap tq, to, tcb, tmn;
+    if (!make_tma_bf16_3d(&tq, Q, D, s.N, BH, kTile) || !make_tma_bf16_3d(&to, O, D, s.N, BH, kTile) ||
+        !make_tma_bf16_3d(&tcb, cb, D, s.M0, s.H, 128) || !make_tma_bf16_3d(&tmn, means, D, s.M0, BH, 128))
+        return cudaErrorInvalidValue;
+    TcAttnParams prm{};
+    prm.BH = BH;
+    prm.H = s.H;
+    prm.N = s.N;
+    prm.M0 = s.M0;
+    prm.M0p = (s.M0 + 15) & ~15;
+    prm.C = 0;
+    prm.P = 0;
+    prm.Mtot = s.M0;
+    prm.ntiles = (s.N + kTile - 1) / kTile;
+    prm.total_tiles = prm.ntiles * BH;
+    prm.sl2 = scale * 1.4426950408889634f;
+    prm.counts = counts;
+    prm.codebook = static_cast<const uint16_t*>(cb);
+    prm.means = static_cast<const uint16_t*>(means);
+    prm.selected = nullptr;
+    prm.status = status;
+    const size_t smem = flat_attn_smem(D, s.M0);
+    auto kern = flat_attention_kernel<D>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    kern<<<std::min(prm.total_tiles, sms), 256, smem, st>>>(tq, to, tcb, tmn, prm);
+    count_launch();
+    return cudaGetLastError();
+}
 
 bool attention_tc_supported(const avq_shape& s, int tile) {
     if (s.dtype != AVQ_BF16 || tile != kTile) return false;

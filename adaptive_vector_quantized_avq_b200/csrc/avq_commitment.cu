@@ -80,8 +80,8 @@ extern "C" int avq_commitment(const avq_shape* s, const void* K, const void* cod
     if (!s) return AVQ_EINVAL;
     if (s->B < 1 || s->H < 1 || s->N < 0 || (s->d != 64 && s->d != 128)) return AVQ_EINVAL;
     if (s->dtype != AVQ_F32 && s->dtype != AVQ_BF16) return AVQ_EINVAL;
-    if (s->M0 < 1 || s->C < 1) return AVQ_EINVAL;
-    if (s->M0 > kMaxM0 || s->C > kMaxC) return AVQ_EUNSUPPORTED;
+    if (s->M0 < 1 || s->C < 0) return AVQ_EINVAL;
+    if (s->M0 > (s->C == 0 ? kMaxFlat : kMaxM0) || s->C > kMaxC) return AVQ_EUNSUPPORTED;
     if ((long long)s->B * s->H * s->N * s->d >= (1LL << 40) || (long long)s->B * s->H > 65535) return AVQ_EUNSUPPORTED;
     const auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
     if (!codebook || !sq_err || (s->N > 0 && (!K || !assign))) return AVQ_EINVAL;

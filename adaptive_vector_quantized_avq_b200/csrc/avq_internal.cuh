@@ -13,6 +13,7 @@ namespace avq {
 // Limits of the on-chip designs (checked by the entry points).
 constexpr int kMaxM0 = 128;
 constexpr int kMaxC = 16;
+constexpr int kMaxFlat = 512;   // codewords of a flat codebook (C == 0)
 
 // Workspace layout: the first 256 bytes are the status block.
 struct StatusBlock {

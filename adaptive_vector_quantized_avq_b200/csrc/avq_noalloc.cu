@@ -72,7 +72,8 @@ extern "C" int avq_attention_noalloc(const avq_shape* s, const void* Q, const vo
     if (!s) return AVQ_EINVAL;
     if (s->B < 1 || s->H < 1 || s->N < 0 || (s->d != 64 && s->d != 128)) return AVQ_EINVAL;
     if (s->dtype != AVQ_F32 && s->dtype != AVQ_BF16) return AVQ_EINVAL;
-    if (s->M0 < 1 || s->C < 1) return AVQ_EINVAL;
+    if (s->M0 < 1 || s->C < 0) return AVQ_EINVAL;
+    if (s->C == 0) return AVQ_EUNSUPPORTED;   // flat codebooks: avq_attention
     if (s->M0 > kMaxM0 || s->C > kMaxC) return AVQ_EUNSUPPORTED;
     if ((long long)s->B * s->H * s->N * s->d >= (1LL << 40)) return AVQ_EUNSUPPORTED;
     if (P < 0 || P > s->M0 || (tile != 64 && tile != 128)) return AVQ_EINVAL;

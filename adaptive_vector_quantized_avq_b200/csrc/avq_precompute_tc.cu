@@ -637,6 +637,307 @@ __global__ void __launch_bounds__(256) precompute_parent_totals_kernel(int BHM0,
     if (lane == 0) counts[prow] += cnt;
 }
 
+// Flat codebook (no children; the codebook is the M0 parents alone) with up
+// to 512 codewords: nearest codeword, counts and value sums (paper §3.2, VQ
+// attention without the tree). The warpgroup pipeline of the tree kernel;
+// the dot products with the codewords come through the warpgroup's 128 TMEM
+// columns in chunks of at most 128 codewords, twice per tile (the minimum,
+// then the codewords within the error bound of it), and a key whose nearest
+// codeword the bound leaves open is listed for the exact decision.
+template <int D, int NWG>
+__global__ void __launch_bounds__(128 * NWG, 1)
+flat_precompute_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmCB,
+                       const TcPreParams p) {
+    constexpr int KH = D / 64;
+    constexpr uint32_t IMG = KH * kRegion;
+    constexpr int KSTEPS = D / 16;
+    constexpr int NT = 128 * NWG;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = align1024p(smem_raw);
+    const int M0c = (p.M0 + 127) & ~127;                    // codeword rows held (whole 128-row boxes)
+    const int nchunks = M0c / 128;
+    uint8_t* sK0 = base;                                     // K stage of warpgroup w: sK0 + w*IMG
+    uint8_t* sB1 = base + NWG * IMG;                         // codewords (K-major, TMA), M0c rows
+    const uint32_t b1_region = (uint32_t)M0c * 128u;         // bytes between its 64-column blocks
+    float* sCn = reinterpret_cast<float*>(sB1 + KH * b1_region);   // [M0c] norms (+inf past M0)
+    float* sRed = sCn + M0c;                                 // [16]
+    int* sCnt = reinterpret_cast<int*>(sRed + 16);           // [M0]
+    int* sFix = sCnt + p.M0;                                 // [1]
+    uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(sFix + 1) + 7) & ~uintptr_t(7));
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 2 * NWG + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = tid >> 7, lt = tid & 127;
+    const int wgbar = 1 + wg;
+    uint64_t* barK = &bars[2 * wg];
+    uint64_t* barM = &bars[2 * wg + 1];
+    uint64_t* barH = &bars[2 * NWG];
+    uint8_t* sK = sK0 + wg * IMG;
+    const int g0 = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
+    const int g1 = (int)(((long long)(blockIdx.x + 1) * p.total_tiles) / gridDim.x);
+
+    if (warp == 0) {
+        tmem_alloc(sTmem, 128 * NWG);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        *sFix = 0;
+        for (int i = 0; i < 2 * NWG + 1; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmCB);
+    }
+    for (int i = tid; i < p.M0; i += NT) sCnt[i] = 0;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sTmem;
+    const uint32_t trow = tmem + 128 * wg + ((uint32_t)((warp & 3) * 32) << 16);
+    const float c_exp = 2.f * (5.f * D + 8.f) * 5.9604644775390625e-08f;
+
+    uint32_t kph = 0, mph = 0, hph = 0;
+    bool failed = false;
+    int cur_bh = -1;
+    float cnmax = 0.f;
+
+    auto issue_k = [&](int g) {
+        const int bh = g / p.ntiles, t = g % p.ntiles;
+        mbar_arrive_expect_tx(barK, IMG);
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh) tma_load_3d(sK + kh * kRegion, &tmK, barK, kh * 64, t * kTile, bh);
+    };
+    auto flush_counts = [&](int bh) {
+        for (int i = tid; i < p.M0; i += NT) {
+            const int c = sCnt[i];
+            if (c) {
+                atomicAdd(p.counts + (size_t)bh * p.Mtot + i, c);
+                sCnt[i] = 0;
+            }
+        }
+    };
+    // MMA of codeword chunk j into this warpgroup's TMEM columns and the wait
+    // for it (thread lt 0 issues; false if a wait ran out)
+    auto chunk_mma = [&](int j, bool& ok) {
+        if (lt == 0 && ok) {
+            const int nj = min(128, ((p.M0 + 15) & ~15) - 128 * j);
+            const uint32_t idesc = idesc_bf16_f32(128, nj, false);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks)
+                mma_ss(tmem + 128 * wg, desc_k128(sK, ks), desc_k128(sB1 + j * 128 * 128, ks, b1_region), idesc,
+                       ks > 0);
+            mma_commit(barM);
+        }
+        ok = mbar_wait(barM, mph) && ok;
+        mph ^= 1;
+        tc_fence_after();
+    };
+
+    for (int gs = g0; gs < g1 && !failed;) {
+        const int bh = gs / p.ntiles, h = bh % p.H;
+        const int ge = min(g1, (bh + 1) * p.ntiles);
+        __syncthreads();
+        if (lt == 0 && gs + wg < ge) issue_k(gs + wg);
+        if (cur_bh >= 0) flush_counts(cur_bh);
+        bool ok = true;
+        if (cur_bh < 0 || h != cur_bh % p.H) {
+            if (tid == 0) {
+                mbar_arrive_expect_tx(barH, KH * (uint32_t)M0c * 128u);
+                for (int kh = 0; kh < KH; ++kh)
+                    for (int r0 = 0; r0 < M0c; r0 += 128)
+                        tma_load_3d(sB1 + kh * b1_region + r0 * 128, &tmCB, barH, kh * 64, r0, h);
+            }
+            ok = mbar_wait(barH, hph);
+            hph ^= 1;
+            float mx = 0.f;
+            for (int i = tid; i < M0c; i += NT) {
+                float cn = INFINITY;
+                if (i < p.M0 && ok) {
+                    cn = norm2_f64<D>(sB1, [&](int j) { return swz_off(i, j, b1_region); });
+                    mx = fmaxf(mx, cn);
+                }
+                sCn[i] = cn;
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) sRed[warp] = mx;
+        }
+        if (__syncthreads_or(!ok)) { failed = true; break; }
+        cnmax = sRed[0];
+        for (int w = 1; w < NT / 32; ++w) cnmax = fmaxf(cnmax, sRed[w]);
+        cur_bh = bh;
+
+        for (int g = gs + wg; g < ge; g += NWG) {
+            const int t = g % p.ntiles;
+            const int rows = min(kTile, p.N - t * kTile);
+            const bool valid = lt < rows;
+            ok = true;
+            if (lt == 0) ok = mbar_wait(barK, kph);
+            kph ^= 1;
+            // pass 1: the smallest v = ||C||^2 - 2 k.C over all chunks
+            float m = INFINITY;
+            for (int j = 0; j < nchunks; ++j) {
+                chunk_mma(j, ok);
+                for (int c = 0; c < 8; ++c) {
+                    const int col = 128 * j + 16 * c;
+                    if (col < ((p.M0 + 15) & ~15)) {
+                        float v16[16];
+                        tmem_ld16f(trow + 16 * c, v16);
+                        tmem_wait_ld();
+                        tmem_touch16f(v16);
+#pragma unroll
+                        for (int q = 0; q < 16; q += 4) {
+                            const float4 cn4 = *reinterpret_cast<const float4*>(sCn + col + q);
+                            m = fmin3(m, fmaf(-2.f, v16[q], cn4.x), fmaf(-2.f, v16[q + 1], cn4.y));
+                            m = fmin3(m, fmaf(-2.f, v16[q + 2], cn4.z), fmaf(-2.f, v16[q + 3], cn4.w));
+                        }
+                    }
+                }
+                tc_fence_before();
+                wg_sync(wgbar);   // the TMEM columns are free for the next chunk
+            }
+            float kn;
+            {
+                float kn0 = 0.f, kn1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < D / 8; ++j) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(sK + swz_off(lt, j));
+                    kn0 = sqacc_lo(w.x, kn0); kn1 = sqacc_hi(w.x, kn1);
+                    kn0 = sqacc_lo(w.y, kn0); kn1 = sqacc_hi(w.y, kn1);
+                    kn0 = sqacc_lo(w.z, kn0); kn1 = sqacc_hi(w.z, kn1);
+                    kn0 = sqacc_lo(w.w, kn0); kn1 = sqacc_hi(w.w, kn1);
+                }
+                kn = __fadd_rn(kn0, kn1);
+            }
+            // pass 2: the codewords within the error band of the smallest
+            // (count in the low 10 bits, their index sum above)
+            const float thr = __fadd_ru(m, 2.f * c_exp * (kn + cnmax));
+            int acc = 0;
+            for (int j = 0; j < nchunks; ++j) {
+                chunk_mma(j, ok);
+                for (int c = 0; c < 8; ++c) {
+                    const int col = 128 * j + 16 * c;
+                    if (col < ((p.M0 + 15) & ~15)) {
+                        float v16[16];
+                        tmem_ld16f(trow + 16 * c, v16);
+                        tmem_wait_ld();
+                        tmem_touch16f(v16);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            if (fmaf(-2.f, v16[q], sCn[col + q]) <= thr) acc += ((col + q) << 10) + 1;
+                    }
+                }
+                tc_fence_before();
+                if (j + 1 < nchunks) wg_sync(wgbar);
+            }
+            const bool one = (acc & 1023) == 1;
+            const int bp = one ? (acc >> 10) : 0;
+            const bool listed = valid && !one;
+            if (wg_sync_or(wgbar, !ok)) { failed = true; break; }   // the K stage and TMEM are free
+            if (lt == 0 && g + NWG < ge) issue_k(g + NWG);
+
+            const int kl = valid ? bp : -1;
+            if (valid) p.assign[(size_t)bh * p.N + t * kTile + lt] = bp;
+            {
+                const unsigned same = __match_any_sync(0xffffffffu, kl);
+                if (valid && lane == __ffs(same) - 1) atomicAdd(&sCnt[bp], __popc(same));
+            }
+            if (listed) {
+                atomicAdd(&p.status->pad[0], 1);
+                const int slot = atomicAdd(sFix, 1);
+                p.fix_list[(size_t)g0 * kTile + slot] = (long long)bh * p.N + (long long)t * kTile + lt;
+            }
+            {
+                const int hl = lane & 15, sub = lane >> 4;
+                constexpr int DPL = D / 16;
+                const size_t row0 = (size_t)bh * p.N + (size_t)t * kTile + 32 * (warp & 3);
+                const uint16_t* vsrc = p.V + row0 * D + hl * DPL;
+                float* vs_lane = p.vsum + (size_t)bh * p.Mtot * D + hl * DPL;
+#pragma unroll 4
+                for (int q = 0; q < 16; ++q) {
+                    const int lfq = __shfl_sync(0xffffffffu, kl, 2 * q + sub);
+                    if (lfq >= 0) {
+                        float* dst = vs_lane + (size_t)lfq * D;
+                        if (D == 64) {
+                            const uint2 w = __ldg(reinterpret_cast<const uint2*>(vsrc + (size_t)(2 * q + sub) * D));
+                            red_v4(dst, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+                        } else {
+                            const uint4 w = __ldg(reinterpret_cast<const uint4*>(vsrc + (size_t)(2 * q + sub) * D));
+                            red_v4(dst, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+                            red_v4(dst + 4, bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+                        }
+                    }
+                }
+            }
+        }
+        if (__syncthreads_or(failed)) { failed = true; break; }
+        gs = ge;
+    }
+
+    __syncthreads();
+    if (!failed && cur_bh >= 0) flush_counts(cur_bh);
+    if (!failed) {
+        const int nf = *sFix;
+        for (int e = warp; e < nf; e += NT / 32)
+            fix_key<D, 0>(p.fix_list[(size_t)g0 * kTile + e], p.K, p.V, p.codebook, p.assign, p.counts, p.vsum,
+                          p.N, p.H, p.M0, p.Mtot);
+    }
+    if (failed && tid == 0) {
+        atomicExch(&p.status->error, (int)AVQ_ETIMEOUT);
+        atomicExch(&p.status->where, (int)blockIdx.x);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128 * NWG);
+    }
+}
+
+size_t flat_smem_bytes(int D, int M0) {
+    const int nwg = D == 64 ? 4 : 2;
+    const size_t M0c = (size_t)((M0 + 127) & ~127);
+    return 1024 + nwg * (size_t)(D / 64) * kRegion + (size_t)(D / 64) * M0c * 128 + M0c * 4 + 16 * 4 +
+           (size_t)M0 * 4 + 4 + 8 + (2 * nwg + 1) * 8 + 16;
+}
+
+template <int D>
+cudaError_t launch_flat_pre(const avq_shape& s, const void* K, const void* V, const void* cb, int32_t* assign,
+                            int32_t* counts, float* vsum, StatusBlock* status, cudaStream_t st) {
+    const int BH = s.B * s.H;
+    CUtensorMap tk, tcb;
+    if (!make_tma_bf16_3d(&tk, K, D, s.N, BH, kTile) || !make_tma_bf16_3d(&tcb, cb, D, s.M0, s.H, 128))
+        return cudaErrorInvalidValue;
+    TcPreParams prm;
+    prm.BH = BH;
+    prm.H = s.H;
+    prm.N = s.N;
+    prm.M0 = s.M0;
+    prm.M0p = (s.M0 + 15) & ~15;
+    prm.Mtot = s.M0;
+    prm.ntiles = (s.N + kTile - 1) / kTile;
+    prm.total_tiles = prm.ntiles * BH;
+    prm.K = static_cast<const uint16_t*>(K);
+    prm.V = static_cast<const uint16_t*>(V);
+    prm.codebook = static_cast<const uint16_t*>(cb);
+    prm.assign = assign;
+    prm.counts = counts;
+    prm.vsum = vsum;
+    prm.status = status;
+    prm.fix_list = reinterpret_cast<long long*>(reinterpret_cast<uint8_t*>(status) + kStatusBytes);
+    constexpr int NWG = D == 64 ? 4 : 2;
+    const size_t smem = flat_smem_bytes(D, s.M0);
+    auto kern = flat_precompute_kernel<D, NWG>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    kern<<<std::min(prm.total_tiles, sms), 128 * NWG, smem, st>>>(tk, tcb, prm);
+    count_launch();
+    return cudaGetLastError();
+}
+
 int pre_nwg(int D) { return D == 64 ? 4 : 2; }
 
 size_t pre_smem_bytes(int D, int M0, int C, int Mtot) {
@@ -696,6 +997,18 @@ cudaError_t launch_pre_tc(const avq_shape& s, const void* K, const void* V, cons
 }
 
 }  // namespace
+
+bool flat_precompute_supported(const avq_shape& s) {
+    return s.dtype == AVQ_BF16 && (s.d == 64 || s.d == 128) && s.C == 0 && s.M0 <= 512 &&
+           flat_smem_bytes(s.d, s.M0) <= 227 * 1024;
+}
+
+cudaError_t launch_flat_precompute(const avq_shape& s, const void* K, const void* V, const void* cb,
+                                   int32_t* assign, int32_t* counts, float* vsum, StatusBlock* status,
+                                   cudaStream_t st) {
+    return s.d == 64 ? launch_flat_pre<64>(s, K, V, cb, assign, counts, vsum, status, st)
+                     : launch_flat_pre<128>(s, K, V, cb, assign, counts, vsum, status, st);
+}
 
 bool precompute_tc_supported(const avq_shape& s) {
     if (s.dtype != AVQ_BF16 || (s.d != 64 && s.d != 128)) return false;

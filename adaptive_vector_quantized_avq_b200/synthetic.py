@@ -132,6 +132,8 @@ WORKLOADS: dict[str, Workload] = {
                  note="maximum length, 256-component Zipf mixture"),
         Workload("refine-d128", 1, 8, 16384, 128, "bf16", 64, 8, (0, 4, 16, 64), 128, 64, None,
                  note="refinement sweep over P at head dim 128"),
+        Workload("flat-512", 1, 16, 16384, 64, "bf16", 512, 0, (0,), 128, 512, None,
+                 note="flat VQ attention (no tree, nothing selected) over 512 codewords"),
     ]
 }
 
@@ -150,10 +152,13 @@ def make_tree_codebook(centres: np.ndarray, M0: int, C: int, child_sigma: float,
                        rng: np.random.Generator) -> np.ndarray:
     """Tree codebook ``[H, M0*(1+C), d]`` (fp64 values on the 2^-5 grid).
 
-    Parents are ``centres[:, :M0]`` moved to the exact mean of their children.
+    Parents are ``centres[:, :M0]`` moved to the exact mean of their children;
+    with C == 0 (a flat codebook) they are the centres on the grid.
     """
     H, _, d = centres.shape
     par = centres[:, :M0, :]                                       # [H, M0, d]
+    if C == 0:
+        return np.clip(np.rint(par / GRID), -_GRID_LIMIT_UNITS, _GRID_LIMIT_UNITS) * GRID
     noise = rng.standard_normal((H, M0, C, d))
     child = par[:, :, None, :] + child_sigma * noise               # [H, M0, C, d]
     units = np.clip(np.rint(child / GRID), -_GRID_LIMIT_UNITS, _GRID_LIMIT_UNITS).astype(np.int64)

@@ -54,7 +54,10 @@ extern "C" {
 typedef enum { AVQ_F32 = 0, AVQ_BF16 = 1 } avq_dtype;
 
 /* Problem sizes. Supported: B, H >= 1; N >= 0; d in {64, 128};
- * 1 <= M0 <= 128; 1 <= C <= 16. */
+ * a tree: 1 <= M0 <= 128, 1 <= C <= 16;
+ * a flat codebook (C == 0, M0 codewords and no children; paper §3.2 VQ
+ * attention): 1 <= M0 <= 512, bf16 only; avq_attention then takes P == 0
+ * and d == 64 with tile 128 (other flat cases return AVQ_EUNSUPPORTED). */
 typedef struct {
     int32_t B, H, N, d;
     int32_t M0, C;
@@ -102,6 +105,7 @@ size_t avq_precompute_workspace_bytes(const avq_shape* s);
  *                                   p*(k) = p (the parent's whole cluster);
  *   counts[b,h,j] / vsum[b,h,j,:] : for a child j, only the keys whose leaf is j.
  * vsum is accumulated in fp32 (summation order unspecified).
+ * With C == 0 the leaf is p*(k) itself: the nearest of the M0 codewords.
  *
  * K, V, codebook: device, read only. assign, counts, vsum: device, written
  * (zeroed by the call). workspace: device, >= avq_precompute_workspace_bytes(s).
@@ -135,6 +139,8 @@ size_t avq_attention_workspace_bytes(const avq_shape* s, int P, int tile);
  *   Zbar_i likewise with counts (the DeltaA correction of papernotes, Key
  *   Designs 3);  O_i = Xbar_i / Zbar_i, stored in Q's dtype.
  * counts/vsum are avq_precompute's outputs for the same codebook.
+ * With C == 0 (a flat codebook) P must be 0 (AVQ_EINVAL otherwise): O is
+ * VQ attention over the M0 codewords, O_i = sum_p e^{S_ip} vsum_p / Zbar_i.
  *
  * Q, codebook, counts, vsum: device, read only. O, selected: device,
  * written. selected may be NULL when P == 0. workspace: device,

@@ -14,6 +14,9 @@ disagrees with something the paper or the mathematics fixes:
 * ``pin_invariants`` -- count/value-sum bookkeeping and score normalisation;
 * ``pin_scale``      -- the logit scale acts as a factor on Q (paper §3.1 writes
                         exp(Q K^T) with any scale folded into Q);
+* ``pin_flat``       -- a flat codebook (no children) is VQ-attention with every
+                        key replaced by its nearest codeword (paper §3.2), by
+                        numpy argmin and dense softmax, and the brute force;
 * ``pin_worked``     -- the worked example's codeword and interaction counts
                         (papernotes summary, "A Worked Example") and Table 1's
                         per-key distance count.
@@ -218,6 +221,23 @@ def pin_scale(orc, seed=11):
         assert np.abs(a["O"] - b["O"]).max() < 1e-12
 
 
+def pin_flat(orc, seed=13):
+    wl = syn.small_workload(N=700, d=16, M0=40, C=0, tile=128, seed=seed, zipf_s=1.1,
+                            n_components=48)
+    inp = syn.generate(wl)
+    K, V, Q, cb = inp.f64("K"), inp.f64("V"), inp.f64("Q"), inp.f64("codebook")
+    assert cb.shape[1] == wl.M0
+    pre = orc.precompute(K, V, cb, wl.M0, 0)
+    nearest, _, _ = _numpy_tree_assignment(K[0, 0], cb[0], wl.M0, 0)
+    assert np.array_equal(nearest, pre["assign"][0, 0]), "flat assignment differs from numpy argmin"
+    assert np.array_equal(np.bincount(nearest, minlength=wl.M0), pre["counts"][0, 0])
+    att = orc.attention(Q, cb, pre["counts"], pre["vsum"], wl.M0, 0, 0, wl.tile, wl.softmax_scale)
+    ref = _dense_softmax_attention(Q[0, 0], cb[0][nearest], V[0, 0], wl.softmax_scale)
+    err = np.abs(att["O_full"][0, 0] - ref).max()
+    assert err < 1e-10, f"flat codebook differs from VQ attention by {err}"
+    pin_brute(orc, cases=[(90, 8, 7, 0, 32, seed), (1, 4, 1, 0, 16, seed + 1)])
+
+
 def pin_worked(orc):
     with open(os.path.join(GOLDEN, "worked_example_64_16_8.json")) as f:
         g = json.load(f)
@@ -234,4 +254,4 @@ def pin_worked(orc):
     assert att["selected"].shape[1] * g["C"] == g["children_per_tile"]
 
 
-ALL_PINS = [pin_brute, pin_p0, pin_pmax, pin_exact, pin_invariants, pin_scale, pin_worked]
+ALL_PINS = [pin_brute, pin_p0, pin_pmax, pin_exact, pin_invariants, pin_scale, pin_flat, pin_worked]

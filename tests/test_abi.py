@@ -44,7 +44,7 @@ def shape(**kw):
 
 
 @pytest.mark.parametrize("bad", [dict(d=32), dict(d=96), dict(B=0), dict(H=0), dict(N=-1),
-                                 dict(M0=0), dict(C=0), dict(dtype=7)])
+                                 dict(M0=0), dict(C=-1), dict(dtype=7), dict(M0=129), dict(C=0, M0=513)])
 def test_workspace_query_rejects_bad_shapes(L, bad):
     assert bd.avq_precompute_workspace_bytes(shape(**bad)) == 0
     assert bd.avq_attention_workspace_bytes(shape(**bad), 2, 128) == 0
@@ -59,6 +59,11 @@ def test_workspace_sizes(L):
     assert bd.avq_attention_workspace_bytes(s, 17, 128) == 0    # P > M0
     assert bd.avq_attention_workspace_bytes(s, -1, 128) == 0
     assert bd.avq_attention_workspace_bytes(s, 4, 96) == 0      # tile not 64/128
+    flat = shape(C=0, M0=512)                                    # a flat codebook of 512 codewords
+    assert bd.avq_precompute_workspace_bytes(flat) >= 256
+    assert bd.avq_attention_workspace_bytes(flat, 0, 128) >= 256 + 1 * 2 * 512 * 64 * 2
+    assert bd.avq_attention_workspace_bytes(flat, 2, 128) == 0   # nothing to select
+    assert bd.avq_attention_workspace_bytes(shape(C=0, M0=512, d=128), 0, 128) == 0   # flat attention: d = 64
 
 
 FAKE = 1 << 40   # 256-byte aligned, never dereferenced: validation fails first

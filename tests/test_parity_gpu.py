@@ -29,6 +29,20 @@ SMALL = [
                                    seed=9, n_components=4), (0, 1, 4)),
     ("one-parent", syn.small_workload(B=1, H=2, N=300, d=64, M0=1, C=1, tile=128, dtype="bf16",
                                       seed=10, n_components=1), (0, 1)),
+    # flat codebooks (C = 0): nearest codeword among up to 512, attention with P = 0
+    ("flat-256", syn.small_workload(B=1, H=2, N=1000, d=64, M0=256, C=0, tile=128, dtype="bf16",
+                                    seed=13, n_components=300), (0,)),
+    ("flat-100-ragged", syn.small_workload(B=2, H=1, N=333, d=64, M0=100, C=0, tile=128,
+                                           dtype="bf16", seed=14, n_components=100, zipf_s=1.1), (0,)),
+    ("flat-512", syn.small_workload(B=1, H=2, N=1500, d=64, M0=512, C=0, tile=128, dtype="bf16",
+                                    seed=15, n_components=600), (0,)),
+    ("flat-3", syn.small_workload(B=1, H=1, N=200, d=64, M0=3, C=0, tile=128, dtype="bf16",
+                                  seed=16, n_components=3), (0,)),
+    # head dim 128: the assignment only (the flat attention kernel is head dim 64)
+    ("flat-d128-512", syn.small_workload(B=1, H=2, N=700, d=128, M0=512, C=0, tile=128,
+                                         dtype="bf16", seed=17, n_components=600), ()),
+    ("flat-d128-200", syn.small_workload(B=2, H=1, N=257, d=128, M0=200, C=0, tile=128,
+                                         dtype="bf16", seed=18, n_components=200), ()),
 ]
 
 
@@ -77,9 +91,9 @@ def _sample_tiles(wl, n=24, seed=0):
     return np.array(sorted(ids))
 
 
-@pytest.mark.parametrize("name", ["tiny-fp32", "vit-b", "long-16k", "max-64k", "refine-d128"])
+@pytest.mark.parametrize("name", ["tiny-fp32", "vit-b", "long-16k", "max-64k", "refine-d128", "flat-512"])
 def test_full_size_parity(lib_built, oracle, name):
-    """The five workloads at full size: assignments/counts/value sums compared
+    """The workloads at full size: assignments/counts/value sums compared
     everywhere, attention on a sample of tiles (plus the first and last)."""
     wl = syn.WORKLOADS[name]
     rep = _run_case(wl, wl.P, oracle, tile_ids_fn=_sample_tiles)
