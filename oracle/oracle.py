@@ -152,6 +152,42 @@ def commitment(K: np.ndarray, codebook: np.ndarray, assign: np.ndarray) -> np.nd
     return out
 
 
+def capture(Q: np.ndarray, K: np.ndarray, assign: np.ndarray, selected: np.ndarray, M0: int, C: int,
+            tile: int, scale: float, rows=None) -> np.ndarray:
+    """Top-P capture of every query (paper §5.2 "Elastic Inference", Table 6,
+    and Figure 7): the share of the query's true softmax attention weight,
+    softmax_k(scale * Q_i . K_k) over all N keys of its (b,h), that falls on
+    keys whose parent is among the P parents selected for the query's tile.
+    A key's parent is its leaf when the leaf is a parent (id < M0), else the
+    parent of that child ((id - M0) // C); ids outside [0, M0*(1+C)) and
+    selected entries outside [0, M0) never count towards the numerator.
+
+    Q, K [B,H,N,d]; assign [B,H,N]; selected [B,H,ceil(N/tile),P].
+    Returns fp64 [B,H,N], or, with ``rows`` (flat indices b*H*N + h*N + i),
+    the values of those queries only."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    B, H, N, d = Q.shape
+    Mtot = M0 * (1 + C)
+    a = np.asarray(assign).reshape(B * H, N).astype(np.int64)
+    parent = np.where(a < M0, a, (a - M0) // max(C, 1))
+    parent = np.where((a >= 0) & (a < Mtot), parent, -1)
+    ntiles = (N + tile - 1) // tile
+    sel = np.asarray(selected).reshape(B * H, ntiles, -1) if N else None
+    Qf, Kf = Q.reshape(B * H, N, d), K.reshape(B * H, N, d)
+    want = np.arange(B * H * N) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros(want.size)
+    for j, r in enumerate(want):
+        bh, i = divmod(int(r), N)
+        s = scale * (Kf[bh] @ Qf[bh, i])                  # logits over all keys
+        w = np.exp(s - s.max())
+        w /= w.sum()                                       # true attention weights
+        chosen = [int(v) for v in sel[bh, i // tile] if 0 <= v < M0]
+        on = np.isin(parent[bh], chosen)
+        out[j] = float(w[on].sum())
+    return out.reshape(B, H, N) if rows is None else out
+
+
 _DEFAULT: Oracle | None = None
 
 

@@ -80,9 +80,11 @@ def test_commitment_gpu(oracle, name):
                                           seed=25, n_components=16),
           "max-64k": syn.WORKLOADS["max-64k"]}[name]
     inp = syn.generate(wl, with_q=False)
-    K, V, cb = (parity.to_device(getattr(inp, n), wl.dtype) for n in ("K", "V", "codebook"))
-    assign, _, _ = bd.precompute(K, V, cb, wl.M0, wl.C)
+    K, cb = (parity.to_device(getattr(inp, n), wl.dtype) for n in ("K", "codebook"))
+    # both sides take the oracle's assignment (no oracle input from the CUDA path)
+    ora_assign = oracle.precompute(inp.f64("K"), inp.f64("V"), inp.f64("codebook"), wl.M0, wl.C)["assign"]
+    assign = torch.from_numpy(np.ascontiguousarray(ora_assign, dtype=np.int32)).cuda()
     got = bd.commitment(K, cb, assign, wl.M0, wl.C).cpu().numpy()
-    ref = orc.commitment(inp.f64("K"), inp.f64("codebook"), assign.cpu().numpy())
+    ref = orc.commitment(inp.f64("K"), inp.f64("codebook"), ora_assign)
     np.testing.assert_allclose(got, ref, rtol=2e-6)
     torch.cuda.synchronize()
