@@ -27,7 +27,7 @@ _STATUS = {0: "AVQ_OK", -1: "AVQ_EINVAL", -2: "AVQ_EUNSUPPORTED", -3: "AVQ_ECUDA
 EXPORTS = ("avq_precompute_workspace_bytes", "avq_precompute", "avq_attention_workspace_bytes",
            "avq_attention", "avq_device_status", "avq_status_string", "avq_version",
            "avq_kernel_launches", "avq_attention_noalloc", "avq_commitment", "avq_gilbert_order",
-           "avq_gather_rows")
+           "avq_gather_rows", "avq_capture_workspace_bytes", "avq_capture")
 
 
 class AVQError(RuntimeError):
@@ -84,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.avq_gilbert_order.restype = i32
         L.avq_gather_rows.argtypes = [shp, vp, vp, vp, vp]
         L.avq_gather_rows.restype = i32
+        L.avq_capture_workspace_bytes.argtypes = [shp, i32, i32]
+        L.avq_capture_workspace_bytes.restype = sz
+        L.avq_capture.argtypes = [shp, vp, vp, vp, vp, i32, i32, ctypes.c_float, vp, vp, sz, vp]
+        L.avq_capture.restype = i32
         L.avq_kernel_launches.argtypes = []
         L.avq_kernel_launches.restype = ctypes.c_uint64
         _LIB = L
@@ -167,6 +171,16 @@ def avq_gilbert_order(rows: int, cols: int, order) -> int:
 
 def avq_gather_rows(shape, src, dst, perm, stream=None) -> int:
     return lib().avq_gather_rows(ctypes.byref(shape), _ptr(src), _ptr(dst), _ptr(perm), _stream(stream))
+
+
+def avq_capture_workspace_bytes(shape, P, tile) -> int:
+    return lib().avq_capture_workspace_bytes(ctypes.byref(shape), P, tile)
+
+
+def avq_capture(shape, Q, K, assign, selected, P, tile, scale, capture, workspace, workspace_bytes,
+                stream=None) -> int:
+    return lib().avq_capture(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(assign), _ptr(selected), P, tile,
+                             float(scale), _ptr(capture), _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def avq_device_status(workspace, stream=None) -> int:
@@ -258,6 +272,38 @@ def commitment(K: torch.Tensor, codebook: torch.Tensor, assign: torch.Tensor, M0
     rc = avq_commitment(make_shape(B, H, N, d, M0, C, K.dtype), K, codebook, assign, out, stream)
     if rc != AVQ_OK:
         raise AVQError(rc, "avq_commitment")
+    return out
+
+
+def capture(Q: torch.Tensor, K: torch.Tensor, assign: torch.Tensor, selected: torch.Tensor | None,
+            M0: int, C: int, P: int, tile: int, scale: float | None = None, *,
+            ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Top-P capture of every query ([B,H,N] fp32): the share of its exact
+    softmax attention weight on keys whose parent is selected for its tile.
+    Raises on a device-side timeout."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    _check(assign, "assign", torch.int32)
+    B, H, N, d = Q.shape
+    if K.shape != Q.shape or assign.shape != (B, H, N):
+        raise ValueError(f"shapes: Q {tuple(Q.shape)}, K {tuple(K.shape)}, assign {tuple(assign.shape)}")
+    if P > 0:
+        _check(selected, "selected", torch.int32)
+        if selected.shape != (B, H, (N + tile - 1) // tile, P):
+            raise ValueError(f"selected has shape {tuple(selected.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    shape = make_shape(B, H, N, d, M0, C, Q.dtype)
+    if ws is None:
+        ws = workspace(avq_capture_workspace_bytes(shape, P, tile), Q.device)
+    out = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    rc = avq_capture(shape, Q, K, assign, selected if P > 0 else None, P, tile, scale, out, ws, ws.numel(),
+                     stream)
+    if rc != AVQ_OK:
+        raise AVQError(rc, "avq_capture")
+    st = avq_device_status(ws, stream)
+    if st != AVQ_OK:
+        raise AVQError(st, "avq_capture (device status)")
     return out
 
 

@@ -200,6 +200,33 @@ int avq_commitment(const avq_shape* s, const void* K, const void* codebook, cons
                    double* sq_err, void* stream);
 
 /*
+ * Top-P capture (paper §5.2 "Elastic Inference via Top-P Adjustment",
+ * Table 6; Figure 7): for every query i of head (b,h), in tile t = i / tile,
+ *   capture[b,h,i] = sum_{k : parent(k) in sel(t)} e^{s_ik} / sum_k e^{s_ik},
+ *   s_ik = scale * Q_i . K_k over ALL N keys of the head (the true, exact
+ *   softmax attention weights),
+ * where parent(k) = assign[b,h,k] if < M0, else (assign[b,h,k] - M0) / C (the
+ * leaf's parent), and sel(t) = selected[b,h,t,0..P-1] (as written by
+ * avq_attention with the same P and tile). Leaf ids outside [0, M0*(1+C))
+ * and selected entries outside [0, M0) count only in the denominator; a
+ * parent listed twice counts once. P == 0 gives 0 everywhere. A diagnostic
+ * off the forward path: it costs an exact-attention pass (N^2 logits per
+ * head, no values), fp32 logits from bf16 products, fp64 running sums.
+ *
+ * Supported: bf16, d in {64, 128}, tile 128 (fp32 inputs and tile 64:
+ * AVQ_EUNSUPPORTED); a flat codebook (C == 0) takes P == 0 only.
+ * Q, K: device [B,H,N,d] read only; assign: device [B,H,N] int32;
+ * selected: device [B,H,ceil(N/tile),P] int32 (may be NULL when P == 0);
+ * capture: device [B,H,N] float32, written. workspace: device,
+ * >= avq_capture_workspace_bytes(s, P, tile) (the status word: a bounded
+ * wait that ran out sets AVQ_ETIMEOUT).
+ */
+size_t avq_capture_workspace_bytes(const avq_shape* s, int P, int tile);
+int avq_capture(const avq_shape* s, const void* Q, const void* K, const int32_t* assign,
+                const int32_t* selected, int P, int tile, float scale, float* capture,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Query reordering along a Gilbert space-filling curve (paper §4.2,
  * "Per-query-tile amortization and adaptivity"; appendix "Spatial reordering
  * ablation", Table 8): tokens laid out on a rows x cols grid (token

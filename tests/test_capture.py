@@ -100,3 +100,89 @@ def test_capture_additive_over_disjoint_selections(oracle):
     np.testing.assert_allclose(cab, ca + cb_, rtol=0, atol=1e-12)
     rep = np.concatenate([a, a[..., :1]], axis=3)
     np.testing.assert_array_equal(orc.capture(Q, K, *args, rep, wl.M0, wl.C, wl.tile, 0.5), ca)
+
+
+def test_capture_argument_errors():
+    """Rejected on the host before any CUDA call (no GPU needed)."""
+    from adaptive_vector_quantized_avq_b200 import binding as bd
+    from adaptive_vector_quantized_avq_b200 import build as bl
+    bl.build()
+    A = 1 << 20   # an aligned address that is never dereferenced
+    ws = bd.avq_capture_workspace_bytes
+    shape = bd.make_shape(1, 2, 300, 64, 16, 4, bd.AVQ_BF16)
+    assert ws(shape, 4, 128) == 256
+    assert ws(shape, 4, 64) == 0                       # 128-query tiles only
+    assert ws(bd.make_shape(1, 2, 300, 64, 16, 4, bd.AVQ_F32), 4, 128) == 0
+    call = lambda s, P=4, tile=128, out=A, w=A, wsb=256, sel=A: bd.avq_capture(
+        s, A, A, A, sel, P, tile, 0.125, out, w, wsb, 0)
+    assert call(shape, out=None) == -1                 # no output
+    assert call(shape, out=A + 2) == -1                # misaligned output
+    assert call(shape, P=17) == -1                     # P > M0
+    assert call(shape, sel=None) == -1                 # P > 0 needs the selection
+    assert call(shape, tile=64) == -2                  # tile 64: not built
+    assert call(shape, wsb=128) == -5                  # workspace too small
+    assert call(bd.make_shape(1, 2, 300, 64, 16, 4, bd.AVQ_F32)) == -2
+    assert call(bd.make_shape(1, 2, 300, 48, 16, 4, bd.AVQ_BF16)) == -1    # d not in {64, 128}
+
+
+# --------------------------------------------------------------------- GPU
+CAPTURE_TOL = 1e-4   # absolute, on a fraction in [0, 1]
+
+
+def _gpu_case(oracle, wl, P, rows=None, seed=0):
+    import torch
+    import parity
+    from adaptive_vector_quantized_avq_b200 import binding as bd
+    inp = syn.generate(wl)
+    Qf, Kf, Vf, cbf = inp.f64("Q"), inp.f64("K"), inp.f64("V"), inp.f64("codebook")
+    pre = oracle.precompute(Kf, Vf, cbf, wl.M0, wl.C)
+    if P > 0:
+        nt = wl.ntiles
+        ids = np.arange(wl.B * wl.H * nt) if rows is None else np.unique(np.asarray(rows) // wl.N * nt +
+                                                                         (np.asarray(rows) % wl.N) // wl.tile)
+        att = oracle.attention(Qf, cbf, pre["counts"], pre["vsum"], wl.M0, wl.C, P, wl.tile,
+                               wl.softmax_scale, tile_ids=ids)
+        sel = np.zeros((wl.B * wl.H * nt, P), np.int32)
+        sel[ids] = att["selected"]
+        sel = sel.reshape(wl.B, wl.H, nt, P)
+    else:
+        sel = np.zeros((wl.B, wl.H, wl.ntiles, 0), np.int32)
+    Q, K = (parity.to_device(getattr(inp, n), wl.dtype) for n in ("Q", "K"))
+    assign = torch.from_numpy(np.ascontiguousarray(pre["assign"], dtype=np.int32)).cuda()
+    selected = torch.from_numpy(np.ascontiguousarray(sel)).cuda()
+    got = bd.capture(Q, K, assign, selected, wl.M0, wl.C, P, wl.tile, wl.softmax_scale).cpu().numpy()
+    torch.cuda.synchronize()
+    ref = orc.capture(Qf, Kf, pre["assign"], sel, wl.M0, wl.C, wl.tile, wl.softmax_scale, rows=rows)
+    g = got.reshape(-1) if rows is None else got.reshape(-1)[np.asarray(rows)]
+    err = np.abs(g - ref.reshape(-1)).max()
+    assert err <= CAPTURE_TOL, f"capture differs by {err}"
+    return err, float(ref.mean())
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,P", [("d64-ragged", 8), ("d128", 4), ("one-tile", 2), ("p0", 0),
+                                    ("pmax", 16)])
+def test_capture_gpu_small(oracle, name, P):
+    wl = {"d64-ragged": syn.small_workload(B=2, H=2, N=1000, d=64, M0=32, C=4, tile=128, dtype="bf16",
+                                           seed=36, n_components=40),
+          "d128": syn.small_workload(B=1, H=2, N=555, d=128, M0=16, C=8, tile=128, dtype="bf16",
+                                     seed=37, n_components=16),
+          "one-tile": syn.small_workload(B=1, H=1, N=100, d=64, M0=4, C=2, tile=128, dtype="bf16",
+                                         seed=38, n_components=4),
+          "p0": syn.small_workload(B=1, H=2, N=300, d=64, M0=16, C=4, tile=128, dtype="bf16",
+                                   seed=39, n_components=16),
+          "pmax": syn.small_workload(B=1, H=2, N=300, d=64, M0=16, C=4, tile=128, dtype="bf16",
+                                     seed=40, n_components=16)}[name]
+    err, mean = _gpu_case(oracle, wl, P)
+    print(name, P, err, mean)
+
+
+@pytest.mark.gpu
+def test_capture_gpu_max64k_sampled(oracle):
+    """The full max-64k workload at its P; 48 sampled queries (with the first
+    and last) compared against the oracle."""
+    wl = syn.WORKLOADS["max-64k"]
+    rng = np.random.default_rng(41)
+    rows = np.unique(np.concatenate([[0, wl.rows - 1], rng.choice(wl.rows, 46, replace=False)]))
+    err, mean = _gpu_case(oracle, wl, wl.P[-1], rows=rows)
+    print("max-64k", err, mean)
