@@ -585,37 +585,49 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 }
 
 // Flat codebook (no children, nothing selected) with up to 512 codewords:
-// VQ attention over all of them (paper §3.2, Eq. 3: softmax weights with a
-// log-count bias, per-codeword value means). The codewords' logits come
-// through TMEM in chunks of at most 128, twice per tile: first for the row
-// maximum m of x_p = scale*log2(e)*S_p + log2 n_p, then for e'_p = 2^(x_p - m),
-// Zbar = sum e'_p and the value contraction Xbar += W_chunk x mean_chunk
-// (MMA3, accumulated in TMEM across the chunks). One CTA of 256 threads per
-// SM; threads r and r + 128 share query row r, each with half of every chunk.
+// VQ attention over all of them (paper §3.2: softmax weights with a
+// log-count bias, per-codeword value means), in one pass over the codewords.
+// They stream in chunks of 128 (codewords and means of a chunk in one of two
+// TMA stages, from L2); per chunk j MMA1 writes S = Q C_j^T to TMEM, each row
+// takes x_p = scale*log2(e)*S_p + log2 n_p, its chunk maximum M_j (the two
+// threads of a row agree on it through shared memory) and the weights
+// e'_p = 2^(x_p - m) as bf16 into TMEM, and MMA3 accumulates
+// Xbar += W_j x mean_j in TMEM. The shift m is the first chunk's maximum and
+// moves only when a later chunk's exceeds it by more than 2^8 (then Xbar and
+// Zbar are rescaled, after the previous MMA3 has completed): the weights stay
+// below 2^8, exact in relative terms in bf16 and fp32, and the common shift
+// cancels in O = Xbar / Zbar. Two CTAs of 256 threads per SM; threads r and
+// r + 128 share query row r, each with half of every chunk.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
 flat_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                       const __grid_constant__ CUtensorMap tmCB, const __grid_constant__ CUtensorMap tmMN,
                       const TcAttnParams p) {
-    constexpr int KH = D / 64;
-    constexpr uint32_t IMG = KH * kRegion;
+    static_assert(D == 64, "one 64-column block per row");
+    constexpr uint32_t IMG = kRegion;
     constexpr int KSTEPS = D / 16;
     constexpr int OD = D / 2;
-    constexpr uint32_t colW = 128, colO = 192;               // TMEM: S 0..127, W 128..191, O 192..
+    constexpr uint32_t colW = 128, colO = 192;               // TMEM: S 0..127, W 128..191, O 192..255
+    constexpr float kLazy = 8.f;                              // shift moves when a maximum exceeds it by this
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = align1024(smem_raw);
+    uint8_t* sQ = base;                                       // Q tile
+    uint8_t* sStage = base + IMG;                             // O staging
+    uint8_t* sCW = base + 2 * IMG;                            // codewords of a chunk (K-major), 2 stages
+    uint8_t* sMN = base + 4 * IMG;                            // their value means (MN-major), 2 stages
     const int M0c = (p.M0 + 127) & ~127;
-    const int nchunks = M0c / 128;
-    uint8_t* const sQ0 = base;                                // two Q stages
-    uint8_t* sStage = base + 2 * IMG;                         // O staging
-    uint8_t* sB1 = base + 3 * IMG;                            // codewords (K-major), M0c rows
-    uint8_t* sMn = sB1 + (size_t)KH * M0c * 128;              // value means (MN-major), M0c rows
-    float* sLb = reinterpret_cast<float*>(sMn + (size_t)KH * M0c * 128);   // [M0c] log2 n (-inf if empty)
-    float* sX = sLb + M0c;                                    // [2][128] row exchange
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 256);   // q0, q1, mma, head
-    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 4);
+    const int nch = M0c / 128;
+    float* sLb = reinterpret_cast<float*>(base + 6 * IMG);   // [M0c] log2 n (-inf if empty or past M0)
+    float* sX = sLb + M0c;                                    // [2][2][128] chunk maxima (by chunk parity)
+    float* sZ = sX + 512;                                     // [2][128] Zbar halves
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sZ + 256);   // Q, chunk stage 0, 1, S, O
+    uint64_t* barQ = bars;
+    uint64_t* barC = bars + 1;
+    uint64_t* barS = bars + 3;
+    uint64_t* barO = bars + 4;
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 5);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int r = tid & 127, hf = tid >> 7, quarter = warp & 3;
     const int g0 = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
     const int g1 = (int)(((long long)(blockIdx.x + 1) * p.total_tiles) / gridDim.x);
@@ -624,7 +636,7 @@ flat_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmO);
@@ -638,136 +650,162 @@ flat_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t idesc3 = idesc_bf16_f32(128, D, true);
     const int M0p = (p.M0 + 15) & ~15;
-    uint32_t qph = 0, mphase = 0, hphase = 0;
+    const int nchunks = (g1 - g0) * nch;                     // chunks this CTA consumes, in order
+    uint32_t qph = 0, sph = 0, oph = 0;
+    int cu = 0;                                               // chunks consumed: stage cu & 1
     bool failed = false;
     int cur_bh = -1;
 
-    auto issue_q = [&](int g, int stage) {
+    auto issue_q = [&](int g) {
         const int bh = g / p.ntiles, t = g % p.ntiles;
-        mbar_arrive_expect_tx(&bars[stage], IMG);
-#pragma unroll
-        for (int kh = 0; kh < KH; ++kh)
-            tma_load_3d(sQ0 + stage * IMG + kh * kRegion, &tmQ, &bars[stage], kh * 64, t * kTile, bh);
+        mbar_arrive_expect_tx(barQ, IMG);
+        tma_load_3d(sQ, &tmQ, barQ, 0, t * kTile, bh);
     };
-    // logits of codeword chunk j (thread 0 issues; every thread waits)
-    auto chunk_logits = [&](int j, int stage, bool& ok) {
-        if (tid == 0 && ok) {
-            const int nj = min(128, M0p - 128 * j);
-            const uint32_t idesc1 = idesc_bf16_f32(128, nj, false);
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < KSTEPS; ++ks)
-                mma_ss(tmem, desc_k(sQ0 + stage * IMG, ks),
-                       smem_desc_sw128(smem_u32(sB1 + j * 16384) + (uint32_t)(ks >> 2) * (uint32_t)M0c * 128u +
-                                           (uint32_t)(ks & 3) * 32u, 16, 1024),
-                       idesc1, ks > 0);
-            mma_commit(&bars[2]);
-        }
-        ok = mbar_wait(&bars[2], mphase) && ok;
-        mphase ^= 1;
+    // chunk c of this CTA's sequence (tile g0 + c / nch, codewords 128 (c % nch) ..) into stage c & 1
+    auto issue_chunk = [&](int c) {
+        const int g = g0 + c / nch, j = c % nch;
+        const int bh = g / p.ntiles;
+        uint64_t* bar = &barC[c & 1];
+        mbar_arrive_expect_tx(bar, 2 * IMG);
+        tma_load_3d(sCW + (c & 1) * IMG, &tmCB, bar, 0, 128 * j, bh % p.H);
+        tma_load_3d(sMN + (c & 1) * IMG, &tmMN, bar, 0, 128 * j, bh);
+    };
+    // (thread 0) MMA1 of chunk c (chunk j of the current tile), once its stage landed
+    auto issue_s = [&](int c, int j, bool& ok) {
+        ok = mbar_wait(&barC[c & 1], (uint32_t)(c >> 1) & 1u) && ok;
+        if (!ok) return;
+        const int nj = min(128, M0p - 128 * j);
+        const uint32_t idesc1 = idesc_bf16_f32(128, nj, false);
         tc_fence_after();
-    };
-    // this thread's 64 columns of the chunk (as x = scale*log2e*S + log2 n; -inf past the codebook)
-    auto load_x = [&](int j, float* x) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int col = 128 * j + 64 * hf + 16 * b;
-            if (col < M0p) tmem_ld16f(trow + 64 * hf + 16 * b, x + 16 * b);
-        }
-        tmem_wait_ld();
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            tmem_touch16f(x + 16 * b);
-            const int col = 128 * j + 64 * hf + 16 * b;
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                x[16 * b + k] = col < M0p ? fmaf(x[16 * b + k], p.sl2, sLb[col + k]) : -INFINITY;
-        }
+        for (int ks = 0; ks < KSTEPS; ++ks)
+            mma_ss(tmem, desc_k(sQ, ks), desc_k(sCW + (c & 1) * IMG, ks), idesc1, ks > 0);
+        mma_commit(barS);
     };
 
-    if (tid == 0 && g0 < g1) issue_q(g0, 0);
-    for (int g = g0, it = 0; g < g1; ++g, ++it) {
-        const int stage = it & 1;
-        const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
-        if (tid == 0) bulk_wait_read_all();
-        bool ok = true;
-        if (bh != cur_bh) {   // head change: codewords, means, log-counts
-            __syncthreads();   // every MMA of the previous head has completed (waited by all)
-            if (tid == 0) {
-                mbar_arrive_expect_tx(&bars[3], 2u * KH * (uint32_t)M0c * 128u);
-                for (int kh = 0; kh < KH; ++kh)
-                    for (int r0 = 0; r0 < M0c; r0 += 128) {
-                        tma_load_3d(sB1 + kh * M0c * 128 + r0 * 128, &tmCB, &bars[3], kh * 64, r0, h);
-                        tma_load_3d(sMn + kh * M0c * 128 + r0 * 128, &tmMN, &bars[3], kh * 64, r0, bh);
-                    }
-            }
+    if (tid == 0 && g0 < g1) {
+        issue_q(g0);
+        issue_chunk(0);
+        if (nchunks > 1) issue_chunk(1);
+    }
+    for (int g = g0; g < g1; ++g) {
+        const int bh = g / p.ntiles, t = g % p.ntiles;
+        if (tid == 0) bulk_wait_read_all();   // the previous O store has read the staging buffer
+        if (bh != cur_bh) {                   // log-counts of this (b,h)
+            __syncthreads();
             for (int i = tid; i < M0c; i += 256) {
                 const int n = i < p.M0 ? __ldg(p.counts + (size_t)bh * p.Mtot + i) : 0;
                 sLb[i] = n > 0 ? __log2f((float)n) : -INFINITY;
             }
-            ok = mbar_wait(&bars[3], hphase);
-            hphase ^= 1;
-            if (__syncthreads_or(!ok)) { failed = true; break; }
+            __syncthreads();
             cur_bh = bh;
         }
+        bool ok = true;
         if (tid == 0) {
-            ok = mbar_wait(&bars[stage], (qph >> stage) & 1u);
-            qph ^= 1u << stage;
-            if (ok && g + 1 < g1) issue_q(g + 1, stage ^ 1);
+            ok = mbar_wait(barQ, qph);
+            if (ok) issue_s(cu, 0, ok);
         }
-        // pass 1: the row maximum
-        float mx = -INFINITY;
-        for (int j = 0; j < nchunks; ++j) {
-            chunk_logits(j, stage, ok);
-            float x[64];
-            load_x(j, x);
-#pragma unroll
-            for (int k = 0; k < 64; k += 2) mx = fmax3(mx, x[k], x[k + 1]);
-            tc_fence_before();
-            __syncthreads();   // S is free for the next chunk
-        }
-        sX[hf * 128 + r] = mx;
-        pair_sync(quarter);
-        const float m = fmaxf(sX[r], sX[128 + r]);
-        pair_sync(quarter);
-        // pass 2: weights, Zbar and the value contraction
-        float2 zp = make_float2(0.f, 0.f);
-        for (int j = 0; j < nchunks; ++j) {
-            chunk_logits(j, stage, ok);   // (its wait also covers the previous chunk's MMA3)
-            float x[64];
-            load_x(j, x);
+        qph ^= 1u;
+        float m = -INFINITY;
+        float2 z0 = make_float2(0.f, 0.f), z1 = make_float2(0.f, 0.f);
+        for (int j = 0; j < nch; ++j, ++cu) {
+            const int s = cu & 1;
+            ok = mbar_wait(barS, sph) && ok;   // MMA1 of this chunk, and every MMA before it
+            sph ^= 1u;
+            tc_fence_after();
+            if (tid == 0) {
+                // the previous chunk's stage is free (its MMA3 preceded this MMA1)
+                if (cu >= 1 && cu + 1 < nchunks) issue_chunk(cu + 1);
+                if (j == nch - 1 && g + 1 < g1) issue_q(g + 1);   // the last MMA1 has read Q
+            }
+            // this half's 64 logits x_p in log2 units with the log-count bias:
+            // first their maximum, then (below) the weights from a second read
+            // of S, so that only 16 of them are live at a time
+            float mx = -INFINITY;
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
+                const int col = 128 * j + 64 * hf + 16 * b;
+                if (col < M0p) {
+                    float x[16];
+                    tmem_ld16f(trow + 64 * hf + 16 * b, x);
+                    tmem_wait_ld();
+                    tmem_touch16f(x);
+#pragma unroll
+                    for (int k = 0; k < 16; k += 4) {
+                        const float4 lb = *reinterpret_cast<const float4*>(sLb + col + k);
+                        mx = fmax3(mx, fmaf(x[k], p.sl2, lb.x), fmaf(x[k + 1], p.sl2, lb.y));
+                        mx = fmax3(mx, fmaf(x[k + 2], p.sl2, lb.z), fmaf(x[k + 3], p.sl2, lb.w));
+                    }
+                }
+            }
+            float* sXj = sX + (j & 1) * 256;
+            sXj[hf * 128 + r] = mx;
+            pair_sync(quarter);
+            const float M = fmaxf(sXj[r], sXj[128 + r]);
+            // the shift moves for a row whose maximum exceeds it by more than
+            // kLazy: its Zbar and Xbar are rescaled (the MMA3s so far have
+            // completed). The TMEM accesses are warp-collective, so a warp takes
+            // them when any of its rows moves, with factor 1 for the others.
+            const bool mv = j > 0 && M > m + kLazy;
+            if (j == 0) m = M;
+            if (__any_sync(0xffffffffu, mv)) {
+                const float f = mv ? ex2(m - M) : 1.f;
+                const float2 f2 = make_float2(f, f);
+                z0 = fmul2(z0, f2);
+                z1 = fmul2(z1, f2);
+#pragma unroll 1
+                for (int c = 0; c < OD / 16; ++c) {
+                    uint32_t u[16];
+                    tmem_ld16(trow + colO + hf * OD + 16 * c, u);
+                    tmem_wait_ld();
+                    tmem_touch16(u);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) u[k] = __float_as_uint(__uint_as_float(u[k]) * f);
+                    tmem_st16(trow + colO + hf * OD + 16 * c, u);
+                }
+                if (mv) m = M;
+            }
+            const float2 sl2v = make_float2(p.sl2, p.sl2);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int col = 128 * j + 64 * hf + 16 * b;
+                if (col >= M0p) break;   // (columns past the codebook are not read by MMA3)
+                float x[16];
+                tmem_ld16f(trow + 64 * hf + 16 * b, x);
+                tmem_wait_ld();
+                tmem_touch16f(x);
                 uint32_t w[8];
 #pragma unroll
                 for (int k = 0; k < 16; k += 2) {
-                    const float e0 = ex2(x[16 * b + k] - m), e1 = ex2(x[16 * b + k + 1] - m);
-                    zp = fadd2(zp, make_float2(e0, e1));
-                    w[k >> 1] = pack_bf16x2(e0, e1);
+                    const float2 lb = *reinterpret_cast<const float2*>(sLb + col + k);
+                    const float2 tt = ffma2(make_float2(x[k], x[k + 1]), sl2v, fadd2(lb, make_float2(-m, -m)));
+                    const float2 e = make_float2(ex2(tt.x), ex2(tt.y));
+                    if ((k >> 1) & 1) z1 = fadd2(z1, e);
+                    else z0 = fadd2(z0, e);
+                    w[k >> 1] = pack_bf16x2(e.x, e.y);
                 }
                 tmem_st8(trow + colW + 32 * hf + 8 * b, w);
             }
             tmem_wait_st();
             tc_fence_before();
             if (__syncthreads_or(!ok)) { failed = true; break; }
-            if (tid == 0) {
+            if (tid == 0) {   // MMA3 of this chunk, then the next chunk's MMA1
                 const int nj = min(128, M0p - 128 * j);
                 tc_fence_after();
                 for (int ks = 0; ks < nj / 16; ++ks)
-                    mma_ts(tmem + colO, tmem + colW + 8 * ks,
-                           smem_desc_sw128(smem_u32(sMn + j * 16384) + (uint32_t)ks * 2048u, (uint32_t)M0c * 128u, 1024),
-                           idesc3, j > 0 || ks > 0);
-                if (j + 1 == nchunks) mma_commit(&bars[2]);
+                    mma_ts(tmem + colO, tmem + colW + 8 * ks, desc_mn(sMN + s * IMG, ks), idesc3, j > 0 || ks > 0);
+                if (j + 1 < nch) issue_s(cu + 1, j + 1, ok);
+                else mma_commit(barO);
             }
         }
         if (failed) break;
-        ok = mbar_wait(&bars[2], mphase) && ok;   // the last MMA3
-        mphase ^= 1;
+        ok = mbar_wait(barO, oph) && ok;   // the last MMA3
+        oph ^= 1u;
         tc_fence_after();
         // epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
-        sX[hf * 128 + r] = zp.x + zp.y;
+        sZ[hf * 128 + r] = (z0.x + z0.y) + (z1.x + z1.y);
         pair_sync(quarter);
-        const float inv = 1.f / (sX[r] + sX[128 + r]);
+        const float inv = 1.f / (sZ[r] + sZ[128 + r]);
         const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
         for (int c = 0; c < OD / 32; ++c) {
@@ -789,8 +827,7 @@ flat_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         tc_fence_before();
         if (__syncthreads_or(!ok)) { failed = true; break; }
         if (tid == 0) {
-#pragma unroll
-            for (int kh = 0; kh < KH; ++kh) tma_store_3d(&tmO, sStage + kh * kRegion, kh * 64, t * kTile, bh);
+            tma_store_3d(&tmO, sStage, 0, t * kTile, bh);
             bulk_commit();
         }
     }
@@ -877,7 +914,7 @@ cudaError_t launch_tc(const avq_shape& s, const void* Q, const void* cb, const i
 
 size_t flat_attn_smem(int D, int M0) {
     const size_t M0c = (size_t)((M0 + 127) & ~127);
-    return 1024 + 3 * (size_t)(D / 64) * kRegion + 2 * (size_t)(D / 64) * M0c * 128 + M0c * 4 + 256 * 4 + 64;
+    return 1024 + 6 * (size_t)(D / 64) * kRegion + M0c * 4 + 768 * 4 + 5 * 8 + 16;
 }
 
 bool flat_attention_supported(const avq_shape& s, int P, int tile) {
@@ -924,7 +961,7 @@ cudaError_t launch_flat_attention(const avq_shape& s, const void* Q, const void*
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kern<<<std::min(prm.total_tiles, sms), 256, smem, st>>>(tq, to, tcb, tmn, prm);
+    kern<<<std::min(prm.total_tiles, 2 * sms), 256, smem, st>>>(tq, to, tcb, tmn, prm);
     count_launch();
     return cudaGetLastError();
 }

@@ -493,6 +493,11 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             uint4 kw[D / 8];
 #pragma unroll
             for (int j = 0; j < D / 8; ++j) kw[j] = *reinterpret_cast<const uint4*>(sK + swz_off(lt, j));
+            // the next K tile is written into this stage by TMA (the async proxy)
+            // once the warpgroup meets below; the proxy fence orders these
+            // shared-memory reads, not yet consumed, before that write (a barrier
+            // alone orders them only against other threads' generic accesses)
+            fence_proxy_async_smem();
             tc_fence_before();   // this tile's TMEM reads before the next MMA into the buffer
             if (wg_sync_or(wgbar, !ok)) { failed = true; break; }   // also: the K stage is free
             if (lt == 0 && g + NWG < ge) issue_k(g + NWG);
@@ -833,6 +838,7 @@ flat_precompute_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             const bool one = (acc & 1023) == 1;
             const int bp = one ? (acc >> 10) : 0;
             const bool listed = valid && !one;
+            fence_proxy_async_smem();   // the K stage's reads before its next TMA write
             if (wg_sync_or(wgbar, !ok)) { failed = true; break; }   // the K stage and TMEM are free
             if (lt == 0 && g + NWG < ge) issue_k(g + NWG);
 
@@ -853,18 +859,40 @@ flat_precompute_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                 const size_t row0 = (size_t)bh * p.N + (size_t)t * kTile + 32 * (warp & 3);
                 const uint16_t* vsrc = p.V + row0 * D + hl * DPL;
                 float* vs_lane = p.vsum + (size_t)bh * p.Mtot * D + hl * DPL;
-#pragma unroll 4
-                for (int q = 0; q < 16; ++q) {
-                    const int lfq = __shfl_sync(0xffffffffu, kl, 2 * q + sub);
-                    if (lfq >= 0) {
-                        float* dst = vs_lane + (size_t)lfq * D;
-                        if (D == 64) {
-                            const uint2 w = __ldg(reinterpret_cast<const uint2*>(vsrc + (size_t)(2 * q + sub) * D));
-                            red_v4(dst, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-                        } else {
-                            const uint4 w = __ldg(reinterpret_cast<const uint4*>(vsrc + (size_t)(2 * q + sub) * D));
-                            red_v4(dst, bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-                            red_v4(dst + 4, bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+                // all sixteen rows' loads first, then the reductions
+                if (D == 64) {
+                    uint2 w[16];
+                    int lf[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        lf[q] = __shfl_sync(0xffffffffu, kl, 2 * q + sub);
+                        w[q] = make_uint2(0u, 0u);
+                        if (lf[q] >= 0) w[q] = __ldg(reinterpret_cast<const uint2*>(vsrc + (size_t)(2 * q + sub) * D));
+                    }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (lf[q] >= 0)
+                            red_v4(vs_lane + (size_t)lf[q] * D, bf_lo(w[q].x), bf_hi(w[q].x), bf_lo(w[q].y),
+                                   bf_hi(w[q].y));
+                } else {
+#pragma unroll
+                    for (int h8 = 0; h8 < 16; h8 += 8) {   // eight rows at a time (registers)
+                        uint4 w[8];
+                        int lf[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            lf[q] = __shfl_sync(0xffffffffu, kl, 2 * (h8 + q) + sub);
+                            w[q] = make_uint4(0u, 0u, 0u, 0u);
+                            if (lf[q] >= 0)
+                                w[q] = __ldg(reinterpret_cast<const uint4*>(vsrc + (size_t)(2 * (h8 + q) + sub) * D));
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (lf[q] >= 0) {
+                                float* dst = vs_lane + (size_t)lf[q] * D;
+                                red_v4(dst, bf_lo(w[q].x), bf_hi(w[q].x), bf_lo(w[q].y), bf_hi(w[q].y));
+                                red_v4(dst + 4, bf_lo(w[q].z), bf_hi(w[q].z), bf_lo(w[q].w), bf_hi(w[q].w));
+                            }
                         }
                     }
                 }

@@ -525,6 +525,56 @@ def ingest_ncu(csv_path: str, workload: str, P: int):
     print(json.dumps(out, indent=1))
 
 
+def run_capture(args):
+    """Times the top-P capture diagnostic (`avq_capture`, an exact-attention
+    pass) on the workload's synthetic inputs, with the assignment and the
+    selection from the forward calls; prints one JSON line of its own (not
+    the benchmark line): ms per call and logits per second."""
+    import torch
+
+    from adaptive_vector_quantized_avq_b200 import binding as bd
+
+    wl = syn.WORKLOADS[args.workload]
+    P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
+    if wl.dtype != "bf16" or wl.C == 0:
+        raise SystemExit("capture needs a bf16 tree workload")
+    dev = torch.device("cuda", 0)
+    inp = syn.generate(wl)
+    K, V, Q, cb = (torch.from_numpy(getattr(inp, n).view(np.int16)).to(dev).view(torch.bfloat16)
+                   for n in ("K", "V", "Q", "codebook"))
+    assign, counts, vsum = bd.precompute(K, V, cb, wl.M0, wl.C)
+    _, sel = bd.attention(Q, cb, counts, vsum, wl.M0, wl.C, P, wl.tile, wl.softmax_scale)
+    shape = bd.make_shape(wl.B, wl.H, wl.N, wl.d, wl.M0, wl.C, Q.dtype)
+    ws = bd.workspace(bd.avq_capture_workspace_bytes(shape, P, wl.tile), dev)
+    out = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        rc = bd.avq_capture(shape, Q, K, assign, sel, P, wl.tile, wl.softmax_scale, out, ws, ws.numel(),
+                            stream.cuda_stream)
+        if rc:
+            raise RuntimeError(f"avq_capture failed: {rc}")
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    if bd.avq_device_status(ws) != 0:
+        raise RuntimeError("avq_capture device status")
+    times = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = float(np.median(times))
+    logits = wl.B * wl.H * wl.N * wl.N
+    print(json.dumps({"metric": "top-P capture logits/s", "workload": args.workload, "P": P,
+                      "ms_per_call": ms, "value": logits / (ms * 1e-3), "unit": "logits/s",
+                      "mean_capture": float(out.mean()), "steps": args.steps, "warmup": args.warmup}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -536,6 +586,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--ingest-ncu", metavar="CSV", help="record DRAM traffic per launch from an ncu CSV")
+    ap.add_argument("--capture", action="store_true",
+                    help="time the top-P capture diagnostic instead (its own JSON line)")
     args = ap.parse_args(argv)
     if args.ingest_ncu:
         wl = syn.WORKLOADS[args.workload]
@@ -544,7 +596,9 @@ def main(argv=None):
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.capture:
+        run_capture(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
