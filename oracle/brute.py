@@ -79,3 +79,84 @@ def brute_force(Q, K, V, cb, M0, C, P, T, scale):
             z = sum(e)
             O.append([sum(e[k] * V[k][j] for k in range(N)) / z for j in range(len(V[0]))])
     return {"parent": parent, "leaf": leaf, "selected": selected, "score": scores, "O": O}
+
+
+def deep_paths(keys, cb, M0, C, L):
+    """Per key, the list of row ids from its level-0 node down to its leaf in a
+    depth-L tree (levels stored one after another; node j of level l has the
+    children j*C + c of level l+1): nearest level-0 node, then each level's
+    nearest child of the current node while it is strictly closer."""
+    offs, acc = [], 0
+    for l in range(L):
+        offs.append(acc)
+        acc += M0 * C ** l
+    out = []
+    for k in keys:
+        dist = [_sqd(k, c) for c in cb]                    # every row of the tree
+        local = min(range(M0), key=lambda p: (dist[p], p))
+        path = [local]
+        for l in range(1, L):
+            kids = [offs[l] + local * C + c for c in range(C)]
+            best = min(kids, key=lambda r: (dist[r], r))
+            if not dist[best] < dist[path[-1]]:
+                break
+            path.append(best)
+            local = best - offs[l]
+        out.append(path)
+    return out
+
+
+def brute_force_deep(Q, K, V, cb, M0, C, L, Ps, T, scale):
+    """One head, a depth-L tree, Ps[l] nodes expanded at level l.
+
+    Per key rather than per codeword: at every stage of a tile each key is
+    represented by one node of its path (its level-0 node at first; the next
+    node of its path once the representing node is expanded). A candidate's
+    importance sums, over the tile's queries and the keys that reached it,
+    their softmax share under the current representation; each query's
+    output is a softmax over the keys with the logits of their final
+    representing nodes. Returns dict(paths, selected (per tile, per level),
+    score (per tile, per level: {row id: importance / rows}), O)."""
+    N = len(K)
+    paths = deep_paths(K, cb, M0, C, L)
+
+    def logit(i, j):
+        return scale * sum(a * b for a, b in zip(Q[i], cb[j]))
+
+    ntiles = (len(Q) + T - 1) // T
+    selected, scores, O = [], [], []
+    for t in range(ntiles):
+        rows = list(range(t * T, min((t + 1) * T, len(Q))))
+        depth_rep = [0] * N                                # index into each key's path
+        cands = list(range(M0))
+        tsel, tscore = [], []
+        for l in range(L - 1):
+            w = {c: 0.0 for c in cands}
+            for i in rows:
+                s = [logit(i, paths[k][depth_rep[k]]) for k in range(N)]
+                m = max(s)
+                e = [math.exp(x - m) for x in s]
+                z = sum(e)
+                for k in range(N):
+                    if len(paths[k]) > l and paths[k][l] in w:
+                        w[paths[k][l]] += math.exp(logit(i, paths[k][l]) - m) / z
+            order = sorted(cands, key=lambda c: (-w[c], c))
+            chosen = order[:Ps[l]]
+            tsel.append(chosen)
+            tscore.append({c: w[c] / len(rows) for c in cands})
+            chosen_set = set(chosen)
+            for k in range(N):
+                if depth_rep[k] == l and len(paths[k]) > l + 1 and paths[k][l] in chosen_set:
+                    depth_rep[k] = l + 1
+            offs_next = sum(M0 * C ** x for x in range(l + 1))
+            offs_cur = offs_next - M0 * C ** l
+            cands = [offs_next + (c - offs_cur) * C + j for c in chosen for j in range(C)]
+        selected.append(tsel)
+        scores.append(tscore)
+        for i in rows:
+            s = [logit(i, paths[k][depth_rep[k]]) for k in range(N)]
+            m = max(s)
+            e = [math.exp(x - m) for x in s]
+            z = sum(e)
+            O.append([sum(e[k] * V[k][j] for k in range(N)) / z for j in range(len(V[0]))])
+    return {"paths": paths, "selected": selected, "score": scores, "O": O}
