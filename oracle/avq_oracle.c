@@ -19,7 +19,7 @@
  *   counts     : [B, H, Mtot]     int64
  *   vsum       : [B, H, Mtot, d]
  *
- * Readings of points the paper leaves open (each is listed in the design doc):
+ * Readings of points the paper leaves open:
  *   - argmin ties go to the lowest index; a child replaces the parent only
  *     when strictly closer ("reassigned if a child is closer than the
  *     (cached) parent distance", paper §4.2);

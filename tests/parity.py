@@ -1,7 +1,7 @@
 """Parity harness: the CUDA path (through the C ABI) against the fp64 oracle.
 
-Acceptance (per the method's statement of tolerances, and readings R14 of
-the design notes):
+Acceptance (the method's tolerances; where selections may differ, only
+inside the 1e-6 tie band below):
 * ``assign`` and ``counts`` bit-exact;
 * ``vsum`` within 1e-5 of the per-codeword sum of |V| (fp32 accumulation);
 * ``selected``: every parent whose normalised oracle score lies more than

@@ -1,6 +1,6 @@
-"""Deeper hierarchies (AVQ-Attention §6 proposes them; the readings are in
-the design notes): the numpy fp64 reference of ``oracle/deep.py`` pinned on
-CPU against the two-level C oracle, a per-key brute force, and the exact
+"""Deeper hierarchies (AVQ-Attention §6 proposes them; the readings taken
+are stated in ``oracle/deep.py``): that numpy fp64 reference pinned on CPU
+against the two-level C oracle, a per-key brute force, and the exact
 special cases."""
 import numpy as np
 import pytest
