@@ -53,3 +53,16 @@ def test_mixture_statistics():
 def test_zipf_weights_heavy_first():
     w = syn._mixture_weights(256, 1.1)
     assert np.all(np.diff(w) < 0) and abs(w.sum() - 1) < 1e-12
+
+
+def test_flat_codebook_is_the_centres_on_the_grid():
+    """C = 0: the codebook is M0 codewords (no children), on the bf16-exact grid,
+    spread over distinct centres (no divide-by-zero fix-up)."""
+    wl = syn.WORKLOADS["flat-512"].with_(N=16, H=2)
+    inp = syn.generate(wl)
+    cb = inp.f64("codebook")
+    assert cb.shape == (2, 512, 64) and wl.Mtot == 512
+    assert np.array_equal(np.rint(cb / syn.GRID) * syn.GRID, cb)
+    assert np.abs(cb).max() <= 3.75
+    assert len(np.unique(cb[0], axis=0)) == 512
+    assert np.array_equal(syn.storage_to_f64(syn.to_storage(cb, "bf16"), "bf16"), cb)
