@@ -157,9 +157,10 @@ int avq_attention(const avq_shape* s, const void* Q, const void* codebook,
  * cudaMalloc, or latency-bound code that cannot afford cudaMalloc's implicit
  * device synchronisation). The paper has no counterpart: this is a property
  * of the library's interface only. Same arguments, results and errors as
- * avq_attention, with no workspace: the scratch lives in a fixed 8 MiB array
- * of device memory owned by the library (on every GPU that loads it, until
- * the process exits).
+ * avq_attention for trees (C >= 1; a flat codebook, C == 0, returns
+ * AVQ_EUNSUPPORTED here: use avq_attention), with no workspace: the scratch
+ * lives in a fixed 8 MiB array of device memory owned by the library (on
+ * every GPU that loads it, until the process exits).
  *
  * - Problems whose scratch, 256 + B*H*M0*(1+C)*d*2 bytes, exceeds 8 MiB are
  *   rejected with AVQ_EWORKSPACE before anything is enqueued.

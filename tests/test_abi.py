@@ -113,6 +113,19 @@ def test_attention_argument_errors(L):
     assert call(wsb=0) == -5
 
 
+def test_flat_codebook_argument_rules(L):
+    """C = 0: attention takes P = 0 only (nothing to select); the no-alloc entry
+    point leaves flat codebooks to avq_attention; all decided on the host."""
+    flat = shape(C=0, M0=256)
+    ws = bd.avq_attention_workspace_bytes(flat, 0, 128)
+    assert bd.avq_attention(flat, FAKE, FAKE, FAKE, FAKE, 2, 128, 0.125, FAKE, FAKE, FAKE, ws,
+                            stream=0) == -1
+    assert bd.avq_attention(shape(C=0, M0=256, d=128), FAKE, FAKE, FAKE, FAKE, 0, 128, 0.125, FAKE,
+                            None, FAKE, ws, stream=0) == -2
+    assert bd.avq_attention_noalloc(flat, FAKE, FAKE, FAKE, FAKE, 0, 128, 0.125, FAKE, None,
+                                    stream=0) == -2
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(bd, "_LIB", None)
     monkeypatch.setattr(bd, "library_path", lambda: str(tmp_path / "nope.so"))
