@@ -1,6 +1,5 @@
 """The C-ABI library without a GPU: it loads, exports every symbol the header
 declares, and rejects bad arguments on the host before touching CUDA."""
-import ctypes
 import os
 import re
 

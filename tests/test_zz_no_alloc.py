@@ -6,7 +6,6 @@ This file is collected last on purpose: if it fails, a run that stops at the
 first failure has already run every other test. It loads the library itself,
 so it also passes alone in a fresh process.
 """
-import numpy as np
 import pytest
 import torch
 
