@@ -174,6 +174,49 @@ def make_tree_codebook(centres: np.ndarray, M0: int, C: int, child_sigma: float,
     return cb
 
 
+def make_deep_codebook(centres: np.ndarray, M0: int, C: int, L: int, child_sigma: float,
+                       rng: np.random.Generator) -> np.ndarray:
+    """Depth-L codebook ``[H, M0*(1+C+...+C^(L-1)), d]`` (fp64 values on the
+    2^-5 grid), levels stored one after another, node j of level l with the
+    children j*C + c of level l+1.
+
+    Level l+1 nodes are drawn around their parents with spread
+    ``child_sigma * 2^-l``; then every node is set to the exact mean of its
+    deepest descendants, so that each node is the exact mean of its children
+    in storage (bf16 included). The deepest nodes' grid units are adjusted
+    first so that every subtree's unit sum divides by its size: a node at
+    level l needs divisibility by C^(L-1-l); the remainder is a multiple of
+    C^(L-2-l) (its child subtrees already divide) and is removed one step of
+    that size at a time from distinct deepest descendants, which keeps every
+    deeper constraint. L = 2 gives the two-level layout."""
+    H, _, d = centres.shape
+    assert L >= 1 and C >= 1
+    nodes = [centres[:, :M0, :]]
+    for l in range(1, L):
+        par = np.repeat(nodes[-1], C, axis=1)
+        nodes.append(par + child_sigma * 2.0 ** (1 - l) * rng.standard_normal(par.shape))
+    headroom = sum(C ** k for k in range(L - 1))              # largest total adjustment of one unit
+    units = np.clip(np.rint(nodes[-1] / GRID), -(_GRID_LIMIT_UNITS - headroom),
+                    _GRID_LIMIT_UNITS - headroom).astype(np.int64)   # [H, M0*C^(L-1), d]
+    for l in range(L - 2, -1, -1):
+        size = C ** (L - 1 - l)                                # deepest nodes under a level-l node
+        step = size // C
+        sub = units.reshape(H, -1, size, d)                    # [H, M0*C^l, size, d] (a view)
+        rem = np.mod(sub.sum(axis=2), size)                    # multiple of step, < size
+        k = rem // step                                        # steps to remove, 0 .. C-1
+        # remove one step from the first k deepest descendants of distinct child subtrees
+        first = np.arange(C) * step                            # the first deepest node of each child subtree
+        take = np.arange(C)[None, None, :, None] < k[:, :, None, :]
+        sub[:, :, first, :] -= step * take
+    assert np.all(np.mod(units.reshape(H, M0, -1, d).sum(axis=2), C ** (L - 1)) == 0)
+    levels = []
+    for l in range(L):
+        size = C ** (L - 1 - l)
+        sums = units.reshape(H, M0 * C ** l, size, d).sum(axis=2)
+        levels.append((sums // size) * GRID)
+    return np.concatenate(levels, axis=1)
+
+
 @dataclass
 class Inputs:
     """Storage-format arrays (fp32, or bf16 as uint16 bits) plus their sizes."""

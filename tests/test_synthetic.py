@@ -66,3 +66,22 @@ def test_flat_codebook_is_the_centres_on_the_grid():
     assert np.abs(cb).max() <= 3.75
     assert len(np.unique(cb[0], axis=0)) == 512
     assert np.array_equal(syn.storage_to_f64(syn.to_storage(cb, "bf16"), "bf16"), cb)
+
+
+def test_deep_codebook_means_exact_at_every_level():
+    """Depth-L codebooks: every node is the exact mean of its C children in
+    storage (bf16 included), on the grid and within range; L = 2 has the
+    two-level layout and constraint."""
+    rng = np.random.default_rng(5)
+    for (M0, C, L, d) in [(4, 2, 3, 8), (8, 8, 3, 16), (3, 4, 4, 8), (16, 4, 2, 8), (2, 3, 1, 4)]:
+        cen = rng.standard_normal((2, M0 + 3, d))
+        cb = syn.make_deep_codebook(cen, M0, C, L, 0.1, np.random.default_rng(1))
+        offs = [sum(M0 * C ** k for k in range(lv)) for lv in range(L + 1)]
+        assert cb.shape == (2, offs[L], d)
+        assert np.array_equal(np.rint(cb / syn.GRID) * syn.GRID, cb) and np.abs(cb).max() <= 3.75
+        assert np.array_equal(syn.storage_to_f64(syn.to_storage(cb, "bf16"), "bf16"), cb)
+        for lv in range(L - 1):
+            par = cb[:, offs[lv]:offs[lv + 1]]
+            kids = cb[:, offs[lv + 1]:offs[lv + 2]].reshape(2, M0 * C ** lv, C, d)
+            assert np.array_equal(par * C, kids.sum(axis=2)), (M0, C, L, lv)
+        assert np.abs(cb[:, :M0] - cen[:, :M0]).max() < 1.0      # parents stay near their centres
