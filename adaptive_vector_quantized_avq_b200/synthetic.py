@@ -97,10 +97,11 @@ class Workload:
     seed: int = 0
     scale: float | None = None   # None -> 1/sqrt(d)
     note: str = field(default="", compare=False)
+    L: int = 2                   # codebook depth (2: parents and children)
 
     @property
     def Mtot(self) -> int:
-        return self.M0 * (1 + self.C)
+        return self.M0 * sum(self.C ** k for k in range(self.L))   # M0 (1 + C) at depth 2
 
     @property
     def rows(self) -> int:
@@ -237,7 +238,10 @@ def generate(wl: Workload, *, with_q: bool = True, with_kv: bool = True) -> Inpu
     s_centre, s_lab_k, s_lab_q, s_k, s_q, s_v, s_cb = ss.spawn(7)
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
     centres = np.random.default_rng(s_centre).standard_normal((H, wl.n_components, d))
-    cb = make_tree_codebook(centres, wl.M0, wl.C, wl.child_sigma, np.random.default_rng(s_cb))
+    if wl.L == 2:
+        cb = make_tree_codebook(centres, wl.M0, wl.C, wl.child_sigma, np.random.default_rng(s_cb))
+    else:
+        cb = make_deep_codebook(centres, wl.M0, wl.C, wl.L, wl.child_sigma, np.random.default_rng(s_cb))
     weights = _mixture_weights(wl.n_components, wl.zipf_s)
 
     def mixture_draw(s_lab, s_pt):
@@ -268,9 +272,9 @@ def generate(wl: Workload, *, with_q: bool = True, with_kv: bool = True) -> Inpu
 def small_workload(N: int = 256, d: int = 8, M0: int = 8, C: int = 4, P=(2,), tile: int = 64,
                    B: int = 1, H: int = 1, dtype: str = "f32", n_components: int | None = None,
                    zipf_s: float | None = None, seed: int = 0, scale: float | None = None,
-                   sigma: float = 0.3) -> Workload:
-    """A small workload for oracle and parity checks."""
-    return Workload(f"small-{B}x{H}x{N}x{d}-{M0}-{C}", B, H, N, d, dtype, M0, C,
+                   sigma: float = 0.3, L: int = 2) -> Workload:
+    """A small workload for oracle and parity checks (L: codebook depth)."""
+    return Workload(f"small-{B}x{H}x{N}x{d}-{M0}-{C}" + (f"-L{L}" if L != 2 else ""), B, H, N, d, dtype, M0, C,
                     tuple(P) if not isinstance(P, int) else (P,), tile,
                     n_components if n_components is not None else M0, zipf_s,
-                    sigma=sigma, seed=seed, scale=scale)
+                    sigma=sigma, seed=seed, scale=scale, L=L)

@@ -85,3 +85,20 @@ def test_deep_codebook_means_exact_at_every_level():
             kids = cb[:, offs[lv + 1]:offs[lv + 2]].reshape(2, M0 * C ** lv, C, d)
             assert np.array_equal(par * C, kids.sum(axis=2)), (M0, C, L, lv)
         assert np.abs(cb[:, :M0] - cen[:, :M0]).max() < 1.0      # parents stay near their centres
+
+
+def test_depth_in_workloads():
+    """L = 2 keeps the two-level inputs bit for bit; L = 3 draws a depth-3
+    codebook of M0 (1 + C + C^2) rows that the deep oracle accepts."""
+    wl2 = syn.small_workload(N=64, d=8, M0=4, C=2, dtype="bf16", seed=7)
+    a, b = syn.generate(wl2), syn.generate(wl2.with_(L=2))
+    assert np.array_equal(a.codebook, b.codebook) and wl2.Mtot == 12
+    wl3 = syn.small_workload(N=300, d=8, M0=4, C=2, dtype="bf16", seed=7, L=3)
+    assert wl3.Mtot == 4 * (1 + 2 + 4)
+    inp = syn.generate(wl3)
+    cb = inp.f64("codebook")
+    assert cb.shape == (1, 28, 8)
+    assert np.array_equal(cb[:, 4:12] * 2, cb[:, 12:28].reshape(1, 8, 2, 8).sum(axis=2))
+    from oracle import deep
+    pre = deep.precompute(inp.f64("K"), inp.f64("V"), cb, 4, 2, 3)
+    assert pre["counts"][0, 0, :4].sum() == 300
