@@ -52,6 +52,19 @@ def test_commitment_zero_when_keys_are_codewords(oracle):
     assert orc.commitment(K, cb, r["assign"])[0, 0] == 0.0
 
 
+def test_flat_commitment_is_the_nearest_codeword_distance(oracle):
+    """C = 0: the assigned codeword is the nearest one, so the loss is the sum
+    of each key's smallest squared distance (a direct numpy minimum)."""
+    wl = syn.small_workload(B=1, H=2, N=250, d=8, M0=12, C=0, seed=26, n_components=12)
+    inp = syn.generate(wl)
+    K, cb = inp.f64("K"), inp.f64("codebook")
+    r = oracle.precompute(K, inp.f64("V"), cb, wl.M0, 0)
+    got = orc.commitment(K, cb, r["assign"])
+    for h in range(2):
+        dmin = ((K[0, h][:, None, :] - cb[h][None, :, :]) ** 2).sum(axis=2).min(axis=1)
+        assert abs(got[0, h] - dmin.sum()) <= 1e-12 * dmin.sum()
+
+
 def test_commitment_argument_errors():
     """Rejected on the host before any CUDA call (no GPU needed)."""
     from adaptive_vector_quantized_avq_b200 import binding as bd
