@@ -12,6 +12,21 @@
 namespace avq {
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int check_shape(const avq_shape* s) {
+    if (!s) return AVQ_EINVAL;
+    if (s->B < 1 || s->H < 1 || s->N < 0) return AVQ_EINVAL;
+    if (s->d != 64 && s->d != 128) return AVQ_EINVAL;
+    if (s->dtype != AVQ_F32 && s->dtype != AVQ_BF16) return AVQ_EINVAL;
+    if (s->M0 < 1 || s->C < 0) return AVQ_EINVAL;
+    // a tree holds up to kMaxM0 parents; a flat codebook (C == 0) up to kMaxFlat codewords
+    if (s->M0 > (s->C == 0 ? kMaxFlat : kMaxM0) || s->C > kMaxC) return AVQ_EUNSUPPORTED;
+    // element counts must fit the kernels' index arithmetic
+    const long long rows = (long long)s->B * s->H * s->N;
+    if (rows * s->d >= (1LL << 40)) return AVQ_EUNSUPPORTED;
+    if ((long long)s->B * s->H > 65535LL * 32) return AVQ_EUNSUPPORTED;
+    return AVQ_OK;
+}
 }  // namespace avq
 
 namespace avq {
@@ -46,21 +61,6 @@ using namespace avq;
 namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
-int check_shape(const avq_shape* s) {
-    if (!s) return AVQ_EINVAL;
-    if (s->B < 1 || s->H < 1 || s->N < 0) return AVQ_EINVAL;
-    if (s->d != 64 && s->d != 128) return AVQ_EINVAL;
-    if (s->dtype != AVQ_F32 && s->dtype != AVQ_BF16) return AVQ_EINVAL;
-    if (s->M0 < 1 || s->C < 0) return AVQ_EINVAL;
-    // a tree holds up to kMaxM0 parents; a flat codebook (C == 0) up to kMaxFlat codewords
-    if (s->M0 > (s->C == 0 ? kMaxFlat : kMaxM0) || s->C > kMaxC) return AVQ_EUNSUPPORTED;
-    // element counts must fit the kernels' index arithmetic
-    const long long rows = (long long)s->B * s->H * s->N;
-    if (rows * s->d >= (1LL << 40)) return AVQ_EUNSUPPORTED;
-    if ((long long)s->B * s->H > 65535LL * 32) return AVQ_EUNSUPPORTED;
-    return AVQ_OK;
-}
 
 int check_ws(const void* ws, size_t have, size_t need) {
     if (need == 0) return AVQ_OK;

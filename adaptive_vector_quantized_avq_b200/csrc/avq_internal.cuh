@@ -29,6 +29,11 @@ __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_
 // Host-side count of kernels enqueued by the library (avq_kernel_launches).
 void count_launch(int n = 1);
 
+// Validation of the problem sizes shared by every entry point: AVQ_OK,
+// AVQ_EINVAL (null, sizes out of range) or AVQ_EUNSUPPORTED (beyond the
+// kernels' on-chip limits or index arithmetic).
+int check_shape(const avq_shape* s);
+
 // ---------------------------------------------------------------- element io
 __device__ __forceinline__ float ld_f32(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float ld_f32(const __nv_bfloat16* p) {

@@ -69,13 +69,9 @@ bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t
 extern "C" int avq_attention_noalloc(const avq_shape* s, const void* Q, const void* codebook,
                                      const int32_t* counts, const float* vsum, int P, int tile, float scale,
                                      void* O, int32_t* selected, int32_t* device_status, void* stream) {
-    if (!s) return AVQ_EINVAL;
-    if (s->B < 1 || s->H < 1 || s->N < 0 || (s->d != 64 && s->d != 128)) return AVQ_EINVAL;
-    if (s->dtype != AVQ_F32 && s->dtype != AVQ_BF16) return AVQ_EINVAL;
-    if (s->M0 < 1 || s->C < 0) return AVQ_EINVAL;
+    const int rc = check_shape(s);   // the same size checks as every entry point
+    if (rc != AVQ_OK) return rc;
     if (s->C == 0) return AVQ_EUNSUPPORTED;   // flat codebooks: avq_attention
-    if (s->M0 > kMaxM0 || s->C > kMaxC) return AVQ_EUNSUPPORTED;
-    if ((long long)s->B * s->H * s->N * s->d >= (1LL << 40)) return AVQ_EUNSUPPORTED;
     if (P < 0 || P > s->M0 || (tile != 64 && tile != 128)) return AVQ_EINVAL;
     if (!(scale > 0.f) || !(scale < 3.0e38f)) return AVQ_EINVAL;
     if (!codebook || !counts || !vsum) return AVQ_EINVAL;
