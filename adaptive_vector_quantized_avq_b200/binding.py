@@ -27,7 +27,8 @@ _STATUS = {0: "AVQ_OK", -1: "AVQ_EINVAL", -2: "AVQ_EUNSUPPORTED", -3: "AVQ_ECUDA
 EXPORTS = ("avq_precompute_workspace_bytes", "avq_precompute", "avq_attention_workspace_bytes",
            "avq_attention", "avq_device_status", "avq_status_string", "avq_version",
            "avq_kernel_launches", "avq_attention_noalloc", "avq_commitment", "avq_gilbert_order",
-           "avq_gather_rows", "avq_capture_workspace_bytes", "avq_capture")
+           "avq_gather_rows", "avq_capture_workspace_bytes", "avq_capture", "avq_precompute_deep",
+           "avq_attention_deep_workspace_bytes", "avq_attention_deep")
 
 
 class AVQError(RuntimeError):
@@ -88,6 +89,13 @@ def lib() -> ctypes.CDLL:
         L.avq_capture_workspace_bytes.restype = sz
         L.avq_capture.argtypes = [shp, vp, vp, vp, vp, i32, i32, ctypes.c_float, vp, vp, sz, vp]
         L.avq_capture.restype = i32
+        L.avq_precompute_deep.argtypes = [shp, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.avq_precompute_deep.restype = i32
+        L.avq_attention_deep_workspace_bytes.argtypes = [shp, i32]
+        L.avq_attention_deep_workspace_bytes.restype = sz
+        L.avq_attention_deep.argtypes = [shp, i32, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp, vp, sz,
+                                         vp]
+        L.avq_attention_deep.restype = i32
         L.avq_kernel_launches.argtypes = []
         L.avq_kernel_launches.restype = ctypes.c_uint64
         _LIB = L
@@ -181,6 +189,24 @@ def avq_capture(shape, Q, K, assign, selected, P, tile, scale, capture, workspac
                 stream=None) -> int:
     return lib().avq_capture(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(assign), _ptr(selected), P, tile,
                              float(scale), _ptr(capture), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def avq_precompute_deep(shape, L, K, V, codebook, assign, counts, vsum, stream=None) -> int:
+    return lib().avq_precompute_deep(ctypes.byref(shape), L, _ptr(K), _ptr(V), _ptr(codebook), _ptr(assign),
+                                     _ptr(counts), _ptr(vsum), _stream(stream))
+
+
+def avq_attention_deep_workspace_bytes(shape, L) -> int:
+    return lib().avq_attention_deep_workspace_bytes(ctypes.byref(shape), L)
+
+
+def avq_attention_deep(shape, L, P, Q, codebook, counts, vsum, tile, scale, O, selected, workspace,
+                       workspace_bytes, stream=None) -> int:
+    """`P`: a sequence of L-1 budgets (marshalled to a host int32 array)."""
+    Pa = (ctypes.c_int32 * max(1, len(P)))(*[int(x) for x in P])
+    return lib().avq_attention_deep(ctypes.byref(shape), L, ctypes.cast(Pa, ctypes.c_void_p), _ptr(Q),
+                                    _ptr(codebook), _ptr(counts), _ptr(vsum), tile, float(scale), _ptr(O),
+                                    _ptr(selected), _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def avq_device_status(workspace, stream=None) -> int:
@@ -330,3 +356,57 @@ def gather_rows(x: torch.Tensor, perm: torch.Tensor, *, stream=None) -> torch.Te
     if rc != AVQ_OK:
         raise AVQError(rc, "avq_gather_rows")
     return y
+
+
+def deep_rows(M0: int, C: int, L: int) -> int:
+    """Rows of a depth-L codebook: M0 (1 + C + ... + C^(L-1))."""
+    return sum(M0 * C ** k for k in range(L))
+
+
+def precompute_deep(K: torch.Tensor, V: torch.Tensor, codebook: torch.Tensor, M0: int, C: int, L: int,
+                    *, out=None, stream=None):
+    """Depth-L assignment and path statistics: (assign, counts, vsum)."""
+    for t, n in ((K, "K"), (V, "V"), (codebook, "codebook")):
+        _check(t, n, K.dtype)
+    B, H, N, d = K.shape
+    Mtot = deep_rows(M0, C, L)
+    if V.shape != K.shape or codebook.shape != (H, Mtot, d):
+        raise ValueError(f"shapes: K {tuple(K.shape)}, codebook {tuple(codebook.shape)} (want [{H},{Mtot},{d}])")
+    shape = make_shape(B, H, N, d, M0, C, K.dtype)
+    dev = K.device
+    if out is None:
+        out = (torch.empty((B, H, N), dtype=torch.int32, device=dev),
+               torch.empty((B, H, Mtot), dtype=torch.int32, device=dev),
+               torch.empty((B, H, Mtot, d), dtype=torch.float32, device=dev))
+    rc = avq_precompute_deep(shape, L, K, V, codebook, *out, stream)
+    if rc != AVQ_OK:
+        raise AVQError(rc, "avq_precompute_deep")
+    return out
+
+
+def attention_deep(Q: torch.Tensor, codebook: torch.Tensor, counts: torch.Tensor, vsum: torch.Tensor,
+                   M0: int, C: int, L: int, P, tile: int, scale: float | None = None, *, out=None,
+                   ws: torch.Tensor | None = None, stream=None):
+    """Depth-L adaptive attention: (O [B,H,N,d], selected [B,H,ntiles,sum(P)])."""
+    _check(Q, "Q")
+    _check(codebook, "codebook", Q.dtype)
+    _check(counts, "counts", torch.int32)
+    _check(vsum, "vsum", torch.float32)
+    B, H, N, d = Q.shape
+    P = [int(x) for x in P]
+    if len(P) != L - 1:
+        raise ValueError("one budget per expanded level (L - 1)")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    shape = make_shape(B, H, N, d, M0, C, Q.dtype)
+    ntiles = (N + tile - 1) // tile
+    dev = Q.device
+    if out is None:
+        out = (torch.empty_like(Q), torch.empty((B, H, ntiles, sum(P)), dtype=torch.int32, device=dev))
+    if ws is None:
+        ws = workspace(avq_attention_deep_workspace_bytes(shape, L), dev)
+    rc = avq_attention_deep(shape, L, P, Q, codebook, counts, vsum, tile, scale, out[0],
+                            out[1] if sum(P) > 0 else None, ws, ws.numel(), stream)
+    if rc != AVQ_OK:
+        raise AVQError(rc, "avq_attention_deep")
+    return out

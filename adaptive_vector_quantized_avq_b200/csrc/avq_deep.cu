@@ -1,0 +1,465 @@
+// avq_deep.cu -- AVQ attention over codebook trees deeper than parent ->
+// child (the extension the paper proposes in §6 "Discussion and Conclusion":
+// every further level adds P*C codes to the attention cost per query and
+// multiplies the codebook's resolution by C).
+//
+// The two-level steps carried down every level:
+//   * layout: M0 nodes at level 0, M0*C^l at level l; node j of level l has
+//     the children j*C + c of level l + 1; rows stored level after level
+//     (depth 2 is the [parents | M0 + p*C + c] layout of avq_precompute);
+//   * assignment (paper §4.2): nearest level-0 node, then level by level the
+//     nearest child of the current node replaces it only when strictly
+//     closer (ties to the lower index at every step); the descent stops at
+//     the first level where no child is closer;
+//   * statistics: every node on a key's path counts the key and sums its
+//     value row (the "parent holds its whole cluster" rule at every level);
+//   * attention (paper §4.3), per query tile, one shift per row (the
+//     largest level-0 log-count logit): level-0 weights, then per expanded
+//     level l the candidates (level 0: every level-0 node; deeper: the
+//     children of the nodes expanded at l - 1) get the importance
+//     sum_i A_ic n_c / Zbar_i with the Zbar of the approximation so far, the
+//     P_l largest are expanded (ties to the lower row id), and every child g
+//     of an expanded node f adds (A_g - A_f) [vsum_g, n_g] to Xbar and Zbar.
+//
+// Both kernels run on CUDA cores. The precompute takes one warp per key and
+// decides every comparison on exact fp64 distances summed in index order,
+// so its decisions are the exact ones by construction. The attention takes
+// one CTA per query tile (one thread per row) with the row's Xbar in
+// registers and the per-candidate weights in shared memory.
+#include <algorithm>
+
+#include "avq_internal.cuh"
+
+namespace avq {
+namespace {
+
+constexpr int kMaxL = 4;       // levels of a tree (level 0 .. 3)
+constexpr int kCand = 128;     // candidates per level held on chip
+constexpr float kRescale = 64.f;   // largest weight exponent (log2) before a row's shift moves
+
+struct DeepTree {
+    int M0, C, L, Mtot;
+    int off[kMaxL + 1];        // first row of each level; off[L] = Mtot
+};
+
+DeepTree make_tree(int M0, int C, int L) {
+    DeepTree t{};
+    t.M0 = M0;
+    t.C = C;
+    t.L = L;
+    long long acc = 0, width = M0;
+    for (int l = 0; l < L; ++l) {
+        t.off[l] = (int)acc;
+        acc += width;
+        width *= C;
+    }
+    t.off[L] = (int)acc;
+    t.Mtot = (int)acc;
+    return t;
+}
+
+long long deep_rows(int M0, int C, int L) {
+    long long acc = 0, width = M0;
+    for (int l = 0; l < L; ++l) {
+        acc += width;
+        width *= C;
+    }
+    return acc;
+}
+
+// lexicographic (distance, index) minimum over the warp
+__device__ __forceinline__ void warp_argmin(double& d, int& i) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const double od = __shfl_xor_sync(0xffffffffu, d, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+        if (od < d || (od == d && oi < i)) {
+            d = od;
+            i = oi;
+        }
+    }
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// One warp per key: lanes split the candidates of each step; every distance
+// is exact_sq_dist (fp64, index order, no fusion). The key's path nodes
+// count it and sum its value row (16-byte vector reductions, lanes over d).
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+deep_precompute_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ cb,
+                       int32_t* __restrict__ assign, int32_t* __restrict__ counts, float* __restrict__ vsum,
+                       long long R, int N, int H, DeepTree t) {
+    const long long key = (long long)(((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (key >= R) return;
+    const long long bh = key / N;
+    const int h = (int)(bh % H);
+    const T* k = K + key * D;
+    const T* cbh = cb + (size_t)h * t.Mtot * D;
+    double best = INFINITY;
+    int bi = t.M0;
+    for (int q = lane; q < t.M0; q += 32) {
+        const double s = exact_sq_dist(k, cbh + (size_t)q * D, D);
+        if (s < best) {
+            best = s;
+            bi = q;
+        }
+    }
+    warp_argmin(best, bi);
+    int local = bi < t.M0 ? bi : 0;   // (only non-finite inputs leave bi == M0)
+    int node = local;
+    int path[kMaxL];
+    int depth = 1;
+    path[0] = node;
+    for (int l = 1; l < t.L; ++l) {
+        double dc = INFINITY;
+        int ci = t.C;
+        for (int c = lane; c < t.C; c += 32) {
+            const double s = exact_sq_dist(k, cbh + (size_t)(t.off[l] + local * t.C + c) * D, D);
+            if (s < dc) {
+                dc = s;
+                ci = c;
+            }
+        }
+        warp_argmin(dc, ci);
+        if (!(ci < t.C && dc < best)) break;   // no child strictly closer: the descent stops
+        best = dc;
+        local = local * t.C + ci;
+        node = t.off[l] + local;
+        path[depth++] = node;
+    }
+    const size_t base = (size_t)bh * t.Mtot;
+    if (lane == 0) {
+        assign[key] = node;
+        for (int i = 0; i < depth; ++i) atomicAdd(counts + base + path[i], 1);
+    }
+    // value row: lane j4 takes elements 4 j4 .. 4 j4 + 3
+    for (int j4 = lane; j4 < D / 4; j4 += 32) {
+        const float a = ld_f32(V + key * D + 4 * j4), b = ld_f32(V + key * D + 4 * j4 + 1);
+        const float c = ld_f32(V + key * D + 4 * j4 + 2), e = ld_f32(V + key * D + 4 * j4 + 3);
+        for (int i = 0; i < depth; ++i) red_add_v4(vsum + (base + path[i]) * D + 4 * j4, a, b, c, e);
+    }
+}
+
+// fp32 value means vsum / n (0 for empty nodes)
+__global__ void deep_means_kernel(const float* __restrict__ vsum, const int32_t* __restrict__ counts,
+                                  float* __restrict__ mean, size_t rows, int d) {
+    const size_t n = rows * (size_t)d;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const int c = __ldg(counts + i / d);
+        mean[i] = c > 0 ? __ldg(vsum + i) / (float)c : 0.f;
+    }
+}
+
+struct DeepAttnArgs {
+    const void* Q;
+    const void* cb;
+    const int32_t* counts;
+    const float* mean;     // [BH, Mtot, D] fp32 means
+    void* O;
+    int32_t* selected;     // [BH, ntiles, sum_l P_l], level after level
+    int N, H, ntiles, Psum;
+    int P[kMaxL];
+    float sl2;             // scale * log2(e)
+    DeepTree t;
+};
+
+// One CTA of KT threads per query tile, thread r owns query row r. Shared
+// memory (padded strides keep both the per-row and the per-candidate access
+// patterns free of bank conflicts):
+//   Qs   [D][KT]            the tile's queries as fp32, transposed
+//   E    [kCand][KT + 1]    e'_c = A_c n_c of the current candidates per row
+//   Ap   [kCand][KT + 1]    A_f of the expanded candidates (by rank) per row
+//   W    [kCand]            importance of the current candidates
+//   cid  [kCand]            candidate row ids;  par [kCand]: rank of a
+//                           candidate's expanded parent;  sel [kCand]: the
+//                           expanded candidates (indices) by rank
+//   Zs   [KT]               Zbar per row (0 for rows past the end)
+template <typename T, int D, int KT>
+__global__ void __launch_bounds__(KT)
+deep_attention_kernel(const DeepAttnArgs a) {
+    extern __shared__ float sm[];
+    constexpr int ES = KT + 1;
+    const DeepTree& t = a.t;
+    const int g = blockIdx.x, bh = g / a.ntiles, tt = g % a.ntiles, h = bh % a.H;
+    const int r = threadIdx.x;
+    const int i = tt * KT + r;
+    const bool valid = i < a.N;
+    float* Qs = sm;                                  // [D][KT]
+    float* E = Qs + D * KT;                          // [kCand][ES]
+    float* Ap = E + kCand * ES;                      // [kCand][ES]
+    float* W = Ap + kCand * ES;                      // [kCand]
+    float* Zs = W + kCand;                           // [KT]
+    int* cid = reinterpret_cast<int*>(Zs + KT);      // [kCand]
+    int* par = cid + kCand;                          // [kCand]
+    int* sel = par + kCand;                          // [kCand]
+    const T* Q = static_cast<const T*>(a.Q);
+    const T* cbh = static_cast<const T*>(a.cb) + (size_t)h * t.Mtot * D;
+    const int32_t* cnt = a.counts + (size_t)bh * t.Mtot;
+    const float* mn = a.mean + (size_t)bh * t.Mtot * D;
+
+    // the tile's queries, transposed (coalesced reads of whole rows)
+    for (int idx = r; idx < KT * D; idx += KT) {
+        const int rr = idx / D, j = idx % D;
+        const int ii = tt * KT + rr;
+        Qs[j * KT + rr] = ii < a.N ? ld_f32(Q + ((size_t)bh * a.N + ii) * D + j) : 0.f;
+    }
+    __syncthreads();
+    auto logit = [&](int row) -> float {   // Q_i . codeword(row), fp32
+        const T* c = cbh + (size_t)row * D;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < D; j += 2) {
+            s0 = fmaf(Qs[j * KT + r], ld_f32(c + j), s0);
+            s1 = fmaf(Qs[(j + 1) * KT + r], ld_f32(c + j + 1), s1);
+        }
+        return s0 + s1;
+    };
+
+    float x[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) x[j] = 0.f;
+    // level 0: log-count logits, the row's shift m, weights e' = 2^(x - m)
+    int ncand = t.M0;
+    float m = -INFINITY;
+    for (int c = 0; c < ncand; ++c) {
+        const int n = __ldg(cnt + c);
+        const float xv = n > 0 ? fmaf(logit(c), a.sl2, __log2f((float)n)) : -INFINITY;
+        E[c * ES + r] = xv;
+        m = fmaxf(m, xv);
+    }
+    float z = 0.f;
+    for (int c = 0; c < ncand; ++c) {
+        const float e = exp2f(E[c * ES + r] - m);   // 0 for empty nodes
+        E[c * ES + r] = e;
+        z += e;
+        const float* mc = mn + (size_t)c * D;
+#pragma unroll
+        for (int j = 0; j < D; ++j) x[j] = fmaf(e, __ldg(mc + j), x[j]);
+    }
+    for (int c = r; c < ncand; c += KT) cid[c] = c;
+    int soff = 0;
+    for (int l = 0; l + 1 < t.L; ++l) {
+        Zs[r] = valid ? z : 0.f;
+        __syncthreads();
+        // importance: sum over the tile's rows of e' / Zbar (Zbar so far)
+        for (int c = r; c < ncand; c += KT) {
+            float w = 0.f;
+            for (int rr = 0; rr < KT; ++rr) {
+                const float zz = Zs[rr];
+                if (zz > 0.f) w += E[c * ES + rr] / zz;
+            }
+            W[c] = w;
+        }
+        __syncthreads();
+        const int P = min(a.P[l], ncand);
+        // rank: larger importance first, ties to the lower row id
+        for (int c = r; c < ncand; c += KT) {
+            int rank = 0;
+            const float wc = W[c];
+            const int ic = cid[c];
+            for (int q = 0; q < ncand; ++q) rank += (W[q] > wc) || (W[q] == wc && cid[q] < ic);
+            if (rank < P) {
+                sel[rank] = c;
+                a.selected[((size_t)bh * a.ntiles + tt) * a.Psum + soff + rank] = ic;
+            }
+        }
+        __syncthreads();
+        // A_f = e'_f / n_f of the expanded candidates, kept while the
+        // candidates are replaced by their children
+        for (int k = 0; k < P; ++k) {
+            const int c = sel[k];
+            const int n = __ldg(cnt + cid[c]);
+            Ap[k * ES + r] = n > 0 ? E[c * ES + r] / (float)n : 0.f;
+        }
+        __syncthreads();   // every row has read the expanded candidates' ids and weights
+        // the next candidates: the children of the expanded ones, in rank order
+        int nid[kCand / 32 + 1];
+        int nn = 0;
+        for (int s = r; s < P * t.C; s += KT) nid[nn++] = t.off[l + 1] + (cid[sel[s / t.C]] - t.off[l]) * t.C + s % t.C;
+        __syncthreads();
+        nn = 0;
+        for (int s = r; s < P * t.C; s += KT) {
+            cid[s] = nid[nn++];
+            par[s] = s / t.C;
+        }
+        __syncthreads();
+        ncand = P * t.C;
+        for (int c = 0; c < ncand; ++c) {
+            const int row = cid[c];
+            const int n = __ldg(cnt + row);
+            float e = 0.f;
+            if (n > 0) {
+                float u = fmaf(logit(row), a.sl2, __log2f((float)n)) - m;
+                if (u > kRescale) {
+                    // a child far above the row's shift: move the shift up by a
+                    // whole number k of octaves and scale everything this row
+                    // holds by 2^-k (exact), so that no weight overflows
+                    const float k = ceilf(u);
+                    const float f = exp2f(-k);
+                    m += k;
+                    u -= k;
+                    z *= f;
+#pragma unroll
+                    for (int j = 0; j < D; ++j) x[j] *= f;
+                    for (int cc = 0; cc < c; ++cc) E[cc * ES + r] *= f;
+                    for (int kk = 0; kk < P; ++kk) Ap[kk * ES + r] *= f;
+                }
+                e = exp2f(u);
+                const float dw = e - Ap[par[c] * ES + r] * (float)n;   // (A_g - A_f) n_g
+                z += dw;
+                const float* mc = mn + (size_t)row * D;
+#pragma unroll
+                for (int j = 0; j < D; ++j) x[j] = fmaf(dw, __ldg(mc + j), x[j]);
+            }
+            E[c * ES + r] = e;
+        }
+        soff += a.P[l];
+        __syncthreads();
+    }
+    if (valid) {
+        const float inv = 1.f / z;
+        T* o = static_cast<T*>(a.O) + ((size_t)bh * a.N + i) * D;
+#pragma unroll
+        for (int j = 0; j < D; ++j) st_elem(o + j, x[j] * inv);
+    }
+}
+
+size_t deep_attn_smem(int D, int KT) {
+    return sizeof(float) * ((size_t)D * KT + 2 * (size_t)kCand * (KT + 1) + kCand + KT) + sizeof(int) * 3 * kCand;
+}
+
+template <typename T, int D>
+cudaError_t launch_deep_pre(const avq_shape& s, const DeepTree& t, const void* K, const void* V, const void* cb,
+                            int32_t* assign, int32_t* counts, float* vsum, cudaStream_t st) {
+    const long long R = (long long)s.B * s.H * s.N;
+    const long long blocks = (R * 32 + 255) / 256;
+    deep_precompute_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
+        static_cast<const T*>(K), static_cast<const T*>(V), static_cast<const T*>(cb), assign, counts, vsum, R, s.N,
+        s.H, t);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <typename T, int D, int KT>
+cudaError_t launch_deep_att(const DeepAttnArgs& a, int tiles, cudaStream_t st) {
+    const size_t smem = deep_attn_smem(D, KT);
+    auto kern = deep_attention_kernel<T, D, KT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)tiles, KT, smem, st>>>(a);
+    count_launch();
+    return cudaGetLastError();
+}
+
+int check_deep(const avq_shape* s, int L) {
+    int rc = check_shape(s);
+    if (rc != AVQ_OK) return rc;
+    if (L < 2 || L > kMaxL || s->C < 1) return AVQ_EINVAL;
+    if (s->M0 > kCand) return AVQ_EUNSUPPORTED;
+    if (deep_rows(s->M0, s->C, L) >= (1LL << 24)) return AVQ_EUNSUPPORTED;
+    if ((long long)s->B * s->H * deep_rows(s->M0, s->C, L) * s->d >= (1LL << 40)) return AVQ_EUNSUPPORTED;
+    return AVQ_OK;
+}
+
+bool aligned_p(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+}  // namespace avq
+
+using namespace avq;
+
+extern "C" {
+
+int avq_precompute_deep(const avq_shape* s, int L, const void* K, const void* V, const void* codebook,
+                        int32_t* assign, int32_t* counts, float* vsum, void* stream) {
+    int rc = check_deep(s, L);
+    if (rc != AVQ_OK) return rc;
+    if (!codebook || !counts || !vsum) return AVQ_EINVAL;
+    if (s->N > 0 && (!K || !V || !assign)) return AVQ_EINVAL;
+    if (!aligned_p(K, 16) || !aligned_p(V, 16) || !aligned_p(codebook, 16) || !aligned_p(vsum, 16) ||
+        !aligned_p(assign, 4) || !aligned_p(counts, 4))
+        return AVQ_EINVAL;
+    const DeepTree t = make_tree(s->M0, s->C, L);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t BH = (size_t)s->B * s->H;
+    if (cudaMemsetAsync(counts, 0, BH * t.Mtot * sizeof(int32_t), st) != cudaSuccess) return AVQ_ECUDA;
+    if (cudaMemsetAsync(vsum, 0, BH * t.Mtot * s->d * sizeof(float), st) != cudaSuccess) return AVQ_ECUDA;
+    if (s->N == 0) return AVQ_OK;
+    cudaError_t e;
+    if (s->dtype == AVQ_BF16)
+        e = s->d == 64 ? launch_deep_pre<__nv_bfloat16, 64>(*s, t, K, V, codebook, assign, counts, vsum, st)
+                       : launch_deep_pre<__nv_bfloat16, 128>(*s, t, K, V, codebook, assign, counts, vsum, st);
+    else
+        e = s->d == 64 ? launch_deep_pre<float, 64>(*s, t, K, V, codebook, assign, counts, vsum, st)
+                       : launch_deep_pre<float, 128>(*s, t, K, V, codebook, assign, counts, vsum, st);
+    return e == cudaSuccess ? AVQ_OK : AVQ_ECUDA;
+}
+
+size_t avq_attention_deep_workspace_bytes(const avq_shape* s, int L) {
+    if (check_deep(s, L) != AVQ_OK) return 0;
+    return kStatusBytes + align256((size_t)s->B * s->H * deep_rows(s->M0, s->C, L) * s->d * sizeof(float));
+}
+
+int avq_attention_deep(const avq_shape* s, int L, const int32_t* P, const void* Q, const void* codebook,
+                       const int32_t* counts, const float* vsum, int tile, float scale, void* O, int32_t* selected,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_deep(s, L);
+    if (rc != AVQ_OK) return rc;
+    if (!P || (tile != 64 && tile != 128)) return AVQ_EINVAL;
+    if (!(scale > 0.f) || !(scale < 3.0e38f)) return AVQ_EINVAL;
+    DeepAttnArgs a{};
+    a.t = make_tree(s->M0, s->C, L);
+    a.Psum = 0;
+    for (int l = 0; l + 1 < L; ++l) {
+        const long long ncand = l == 0 ? s->M0 : (long long)P[l - 1] * s->C;
+        if (P[l] < 0 || P[l] > ncand || (long long)P[l] * s->C > kCand) return AVQ_EINVAL;
+        a.P[l] = P[l];
+        a.Psum += P[l];
+    }
+    if (!codebook || !counts || !vsum) return AVQ_EINVAL;
+    if (s->N > 0 && (!Q || !O || (a.Psum > 0 && !selected))) return AVQ_EINVAL;
+    if (!aligned_p(Q, 16) || !aligned_p(O, 16) || !aligned_p(codebook, 16) || !aligned_p(vsum, 16) ||
+        !aligned_p(counts, 4) || !aligned_p(selected, 4))
+        return AVQ_EINVAL;
+    const size_t need = avq_attention_deep_workspace_bytes(s, L);
+    if (!workspace || workspace_bytes < need) return AVQ_EWORKSPACE;
+    if (!aligned_p(workspace, 256)) return AVQ_EINVAL;
+    if (s->N == 0) return AVQ_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* means = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+    const size_t rows = (size_t)s->B * s->H * a.t.Mtot;
+    deep_means_kernel<<<(unsigned)std::min<size_t>((rows * s->d + 255) / 256, 4096), 256, 0, st>>>(vsum, counts,
+                                                                                                    means, rows, s->d);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return AVQ_ECUDA;
+    a.Q = Q;
+    a.cb = codebook;
+    a.counts = counts;
+    a.mean = means;
+    a.O = O;
+    a.selected = selected;
+    a.N = s->N;
+    a.H = s->H;
+    a.ntiles = (s->N + tile - 1) / tile;
+    a.sl2 = scale * 1.4426950408889634f;
+    const int tiles = s->B * s->H * a.ntiles;
+    cudaError_t e;
+#define AVQ_DEEP_CASE(TT, DD, KK) \
+    if (s->d == DD && tile == KK) e = launch_deep_att<TT, DD, KK>(a, tiles, st);
+    if (s->dtype == AVQ_BF16) {
+        AVQ_DEEP_CASE(__nv_bfloat16, 64, 64) AVQ_DEEP_CASE(__nv_bfloat16, 64, 128)
+        AVQ_DEEP_CASE(__nv_bfloat16, 128, 64) AVQ_DEEP_CASE(__nv_bfloat16, 128, 128)
+    } else {
+        AVQ_DEEP_CASE(float, 64, 64) AVQ_DEEP_CASE(float, 64, 128)
+        AVQ_DEEP_CASE(float, 128, 64) AVQ_DEEP_CASE(float, 128, 128)
+    }
+#undef AVQ_DEEP_CASE
+    return e == cudaSuccess ? AVQ_OK : AVQ_ECUDA;
+}
+
+}  // extern "C"

@@ -135,6 +135,8 @@ WORKLOADS: dict[str, Workload] = {
                  note="refinement sweep over P at head dim 128"),
         Workload("flat-512", 1, 16, 16384, 64, "bf16", 512, 0, (0,), 128, 512, None,
                  note="flat VQ attention (no tree, nothing selected) over 512 codewords"),
+        Workload("deep3-16k", 1, 8, 16384, 64, "bf16", 64, 4, ((8, 16),), 128, 64, None,
+                 note="depth-3 tree (64 / 256 / 1024 nodes), 8 then 16 nodes expanded per tile", L=3),
     ]
 }
 

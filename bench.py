@@ -51,17 +51,57 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def algorithmic(wl: syn.Workload, P: int):
+def algorithmic(wl: syn.Workload, P):
     """Per-call algorithmic bytes and tensor FLOPs (paper Table 1 cost model):
     precompute reads K and V and evaluates M0 + C distances per key;
     attention reads Q, writes O and evaluates M0 + P*C logits and weighted
-    sums per query."""
+    sums per query. A depth-L tree (P one budget per expanded level) takes
+    M0 + (L-1) C distances per key and M0 + C sum_l P_l logits per query."""
     s = 2 if wl.dtype == "bf16" else 4
     R, d = wl.rows, wl.d
+    if wl.L > 2:
+        dist = wl.M0 + (wl.L - 1) * wl.C
+        logits = wl.M0 + wl.C * sum(P)
+    else:
+        dist = wl.M0 + wl.C
+        logits = wl.M0 + P * wl.C
     return {
-        "precompute": {"bytes": 2 * R * d * s, "flops": 2 * R * (wl.M0 + wl.C) * d},
-        "attention": {"bytes": 2 * R * d * s, "flops": 4 * R * (wl.M0 + P * wl.C) * d},
+        "precompute": {"bytes": 2 * R * d * s, "flops": 2 * R * dist * d},
+        "attention": {"bytes": 2 * R * d * s, "flops": 4 * R * logits * d},
     }
+
+
+def default_P(wl: syn.Workload, P_arg=None):
+    """The refinement budget a run uses: --P, else the workload's default
+    (the largest of refine-d128's sweep; the per-level tuple of a deep tree)."""
+    if wl.L > 2:
+        return tuple(wl.P[0])
+    if P_arg is not None:
+        return P_arg
+    return wl.P[-1 if wl.name == "refine-d128" else 0]
+
+
+def n_selected(P) -> int:
+    return sum(P) if isinstance(P, tuple) else P
+
+
+def call_precompute(bd, wl, shape, K, V, cb, assign, counts, vsum, ws, stream):
+    if wl.L > 2:
+        return bd.avq_precompute_deep(shape, wl.L, K, V, cb, assign, counts, vsum, stream)
+    return bd.avq_precompute(shape, K, V, cb, assign, counts, vsum, ws, ws.numel(), stream)
+
+
+def call_attention(bd, wl, shape, Q, cb, counts, vsum, P, scale, O, sel, ws, stream):
+    if wl.L > 2:
+        return bd.avq_attention_deep(shape, wl.L, P, Q, cb, counts, vsum, wl.tile, scale, O, sel, ws, ws.numel(),
+                                     stream)
+    return bd.avq_attention(shape, Q, cb, counts, vsum, P, wl.tile, scale, O, sel, ws, ws.numel(), stream)
+
+
+def attention_ws_bytes(bd, wl, shape, P) -> int:
+    if wl.L > 2:
+        return bd.avq_attention_deep_workspace_bytes(shape, wl.L)
+    return bd.avq_attention_workspace_bytes(shape, P, wl.tile)
 
 
 def roofline_for(kind, alg, ms, peaks, sustained):
@@ -180,31 +220,46 @@ class OracleSampler:
     attention with that sequence's statistics), as many as fit the time budget;
     when even one sequence does not fit, the first whole tiles of one. Inputs
     and the statistics the attention reads are prepared untimed, like inputs
-    already resident."""
+    already resident. A depth-L tree uses the numpy depth-L oracle."""
 
-    def __init__(self, wl: syn.Workload, P: int):
-        from oracle import oracle as orc
-        self.O = orc.get()
-        self.threads = self.O.max_threads()
+    def __init__(self, wl: syn.Workload, P):
         self.wl, self.P = wl, P
+        if wl.L > 2:
+            from oracle import deep
+            self.deep = deep
+            self.threads = 1
+        else:
+            from oracle import oracle as orc
+            self.O = orc.get()
+            self.deep = None
+            self.threads = self.O.max_threads()
         self.one = wl.with_(B=1, H=1)
         self.ntiles = self.one.ntiles
         self.heads = [self._head(0)]
         self.n_heads, self.n_tiles = 1, self.ntiles
 
+    def _pre(self, K, V, cb):
+        wl = self.wl
+        if self.deep is not None:
+            return self.deep.precompute(K, V, cb, wl.M0, wl.C, wl.L)
+        return self.O.precompute(K, V, cb, wl.M0, wl.C, nthreads=self.threads)
+
     def _head(self, i: int):
         inp = syn.generate(self.one.with_(seed=self.wl.seed + 7919 * i))
         K, V, Q, cb = (inp.f64(n) for n in ("K", "V", "Q", "codebook"))
-        full = self.O.precompute(K, V, cb, self.wl.M0, self.wl.C, nthreads=self.threads)
-        return K, V, Q, cb, full
+        return K, V, Q, cb, self._pre(K, V, cb)
 
     def _one(self, h, n_tiles: int) -> int:
         wl = self.wl
         K, V, Q, cb, full = h
         n = min(wl.N, n_tiles * wl.tile)
-        self.O.precompute(K[:, :, :n], V[:, :, :n], cb, wl.M0, wl.C, nthreads=self.threads)
-        self.O.attention(Q, cb, full["counts"], full["vsum"], wl.M0, wl.C, self.P, wl.tile,
-                         wl.softmax_scale, tile_ids=np.arange(n_tiles), nthreads=self.threads)
+        self._pre(K[:, :, :n], V[:, :, :n], cb)
+        if self.deep is not None:
+            self.deep.attention(Q, cb, full["counts"], full["vsum"], wl.M0, wl.C, wl.L, self.P, wl.tile,
+                                wl.softmax_scale, tile_ids=np.arange(n_tiles))
+        else:
+            self.O.attention(Q, cb, full["counts"], full["vsum"], wl.M0, wl.C, self.P, wl.tile,
+                             wl.softmax_scale, tile_ids=np.arange(n_tiles), nthreads=self.threads)
         return n
 
     def plan(self, seconds: float) -> None:
@@ -236,6 +291,8 @@ class OracleSampler:
             n = min(wl.N, self.n_tiles * wl.tile)
             what = (f"{n} keys precomputed + {n} queries attended ({self.n_tiles} tiles of {wl.tile}) "
                     f"of one (b,h) sequence of {wl.name}")
+        if self.deep is not None:
+            return f"{what}; fp64 depth-L oracle (numpy, one thread)"
         return f"{what}; fp64 oracle, {self.threads} OpenMP threads"
 
 
@@ -256,7 +313,7 @@ def run_ours(args):
         mg.init("nccl", dev)
 
     wl = syn.WORKLOADS[args.workload]
-    P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
+    P = default_P(wl, args.P)
     wl_rank = mg.rank_workload(wl, rank)
     inp = syn.generate(wl_rank)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -290,11 +347,11 @@ def run_ours(args):
     counts = torch.empty((B, H, Mtot), dtype=torch.int32, device=dev)
     vsum = torch.empty((B, H, Mtot, d), dtype=torch.float32, device=dev)
     O = torch.empty_like(Q)
-    Pmax = max(max(wl.P), P)
+    sweep_P = list(wl.P) if (wl.L == 2 and len(wl.P) > 1) else []
+    Pmax = max([n_selected(P)] + sweep_P)
     sel_buf = torch.empty((B, H, wl.ntiles, max(Pmax, 1)), dtype=torch.int32, device=dev)
-    ws_pre = bd.workspace(bd.avq_precompute_workspace_bytes(shape), dev)
-    ws_att = bd.workspace(max(bd.avq_attention_workspace_bytes(shape, p_, wl.tile) for p_ in set(wl.P) | {P}),
-                          dev)
+    ws_pre = bd.workspace(bd.avq_precompute_workspace_bytes(shape) if wl.L == 2 else 256, dev)
+    ws_att = bd.workspace(max(attention_ws_bytes(bd, wl, shape, p_) for p_ in sweep_P + [P]), dev)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     scale = wl.softmax_scale
@@ -304,14 +361,14 @@ def run_ours(args):
     def step(i, P_, ev=None):
         ncalls[0] += 1
         Ki, Vi, Qi = sets[i % nrot]
-        sel = sel_buf[..., :P_] if P_ > 0 else None
+        k_ = n_selected(P_)
+        sel = sel_buf[..., :k_] if k_ > 0 else None
         if ev is not None:
             ev[0].record(stream)
-        rc = bd.avq_precompute(shape, Ki, Vi, cb, assign, counts, vsum, ws_pre, ws_pre.numel(), sp)
+        rc = call_precompute(bd, wl, shape, Ki, Vi, cb, assign, counts, vsum, ws_pre, sp)
         if ev is not None:
             ev[1].record(stream)
-        rc2 = bd.avq_attention(shape, Qi, cb, counts, vsum, P_, wl.tile, scale, O,
-                               sel, ws_att, ws_att.numel(), sp)
+        rc2 = call_attention(bd, wl, shape, Qi, cb, counts, vsum, P_, scale, O, sel, ws_att, sp)
         if ev is not None:
             ev[2].record(stream)
         if rc or rc2:
@@ -355,8 +412,8 @@ def run_ours(args):
     # throughput against the refinement budget (a workload that lists several
     # P): the same step timed at each of them
     sweep = []
-    if len(wl.P) > 1:
-        for P_ in wl.P:
+    if sweep_P:
+        for P_ in sweep_P:
             for i in range(args.warmup):
                 step(i, P_)
             t_, pre_, att_, _ = timed(P_, args.steps)
@@ -376,8 +433,9 @@ def run_ours(args):
     # output comes down (the two copy directions overlap on the link).
     hK, hV, hQ, hcb = (pinned(getattr(inp, n)) for n in ("K", "V", "Q", "codebook"))
     hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-    sel = sel_buf[..., :P].contiguous() if P > 0 else None
-    hsel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory() if P > 0 else None
+    nsel = n_selected(P)
+    sel = sel_buf[..., :nsel].contiguous() if nsel > 0 else None
+    hsel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory() if nsel > 0 else None
     e2e_steps = max(3, min(args.steps, 20))
     along_b = B > 1
     n_units = B if along_b else H
@@ -388,8 +446,8 @@ def run_ours(args):
     for i in range(n_chunks):
         u = bounds[i + 1] - bounds[i]
         cshape = bd.make_shape(u if along_b else 1, H if along_b else u, N, d, wl.M0, wl.C, tdt)
-        ws_chunks.append((cshape, bd.workspace(bd.avq_precompute_workspace_bytes(cshape), dev),
-                          bd.workspace(bd.avq_attention_workspace_bytes(cshape, P, wl.tile), dev)))
+        ws_chunks.append((cshape, bd.workspace(bd.avq_precompute_workspace_bytes(cshape) if wl.L == 2 else 256, dev),
+                          bd.workspace(attention_ws_bytes(bd, wl, cshape, P), dev)))
 
     def sl(t, i):
         a, b_ = bounds[i], bounds[i + 1]
@@ -411,15 +469,15 @@ def run_ours(args):
                     sl(d_, i).view(h_.dtype).copy_(sl(h_, i), non_blocking=True)
                 hc = (slice(None),) if along_b else (slice(bounds[i], bounds[i + 1]),)
                 cbi = cb if along_b else cb[hc]
-                sel_i = sl(sel, i) if P > 0 else None
-                rc = bd.avq_precompute(cshape, sl(K, i), sl(V, i), cbi, sl(assign, i), sl(counts, i),
-                                       sl(vsum, i), wsp, wsp.numel(), s_.cuda_stream)
-                rc2 = bd.avq_attention(cshape, sl(Q, i), cbi, sl(counts, i), sl(vsum, i), P, wl.tile,
-                                       scale, sl(O, i), sel_i, wsa, wsa.numel(), s_.cuda_stream)
+                sel_i = sl(sel, i) if nsel > 0 else None
+                rc = call_precompute(bd, wl, cshape, sl(K, i), sl(V, i), cbi, sl(assign, i), sl(counts, i),
+                                     sl(vsum, i), wsp, s_.cuda_stream)
+                rc2 = call_attention(bd, wl, cshape, sl(Q, i), cbi, sl(counts, i), sl(vsum, i), P, scale,
+                                     sl(O, i), sel_i, wsa, s_.cuda_stream)
                 if rc or rc2:
                     raise RuntimeError(f"avq call failed: {rc} {rc2}")
                 sl(hO, i).copy_(sl(O, i), non_blocking=True)
-                if P > 0:
+                if nsel > 0:
                     sl(hsel, i).copy_(sel_i, non_blocking=True)
         for s_ in streams:
             stream.wait_stream(s_)
@@ -441,7 +499,7 @@ def run_ours(args):
             raise RuntimeError("device status error in the end-to-end run")
     barrier()
     h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ, hcb))
-    d2h = hO.numel() * hO.element_size() + (hsel.numel() * hsel.element_size() if P > 0 else 0)
+    d2h = hO.numel() * hO.element_size() + (hsel.numel() * hsel.element_size() if nsel > 0 else 0)
 
     # max over ranks
     ms_total, e2e_ms, pre_avg, att_avg = mg.max_over_ranks(
@@ -473,7 +531,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": wl.name, "B": B, "H": H, "N": N, "d": d, "M0": wl.M0,
                        "C": wl.C, "P": P, "tile": wl.tile, "scale": scale,
-                       "query_rows_per_gpu": wl.rows, "l2": l2_note,
+                       "query_rows_per_gpu": wl.rows, "l2": l2_note, **({"L": wl.L} if wl.L > 2 else {}),
                        "seed": f"{wl.seed}+rank"},
             "kernels": {k: {"ms_avg": kern[k], "ms_min": min(pre_ms if k == 'precompute' else att_ms),
                             "roofline": rl[k]} for k in kern},
@@ -512,7 +570,7 @@ def run_reference(args):
     if rank != 0:
         return
     wl = syn.WORKLOADS[args.workload]
-    P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
+    P = default_P(wl, args.P)
     smp = OracleSampler(wl, P)
     per_step = 150.0 / max(1, args.steps + args.warmup)
     smp.plan(per_step)                    # calibration and input preparation, untimed
@@ -584,8 +642,8 @@ def run_capture(args):
     from adaptive_vector_quantized_avq_b200 import binding as bd
 
     wl = syn.WORKLOADS[args.workload]
-    P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
-    if wl.dtype != "bf16" or wl.C == 0:
+    P = default_P(wl, args.P)
+    if wl.dtype != "bf16" or wl.C == 0 or wl.L != 2:
         raise SystemExit("capture needs a bf16 tree workload")
     dev = torch.device("cuda", 0)
     inp = syn.generate(wl)
@@ -640,7 +698,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.ingest_ncu:
         wl = syn.WORKLOADS[args.workload]
-        P = args.P if args.P is not None else wl.P[-1 if args.workload == "refine-d128" else 0]
+        P = default_P(wl, args.P)
         ingest_ncu(args.ingest_ncu, args.workload, P)
         return
     if args.warmup < 3:

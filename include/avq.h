@@ -254,6 +254,51 @@ int avq_gilbert_order(int rows, int cols, int32_t* order);
 int avq_gather_rows(const avq_shape* s, const void* src, void* dst, const int32_t* perm, void* stream);
 
 /*
+ * Deeper codebook trees (paper §6 "Discussion and Conclusion": each further
+ * level adds P*C codes to the attention cost per query and multiplies the
+ * codebook's resolution by C; the pages propose it without testing it). The
+ * two-level steps carried down every level of a depth-L tree:
+ *
+ *   codebook : [H, Mtot, d], Mtot = M0 (1 + C + ... + C^(L-1)); level l holds
+ *              M0 C^l rows, stored level after level; node j of level l has
+ *              the children j C + c (c < C) of level l + 1 (depth 2 is the
+ *              avq_precompute layout). s->M0 = level-0 nodes, s->C = branching.
+ *
+ * avq_precompute_deep (paper §4.2 carried down): nearest level-0 node, then
+ * level by level the nearest child of the current node replaces it only when
+ * STRICTLY closer (ties to the lower index at every step); the descent stops
+ * at the first level where no child is closer; assign = the last node's row.
+ * Every node on a key's path counts the key and sums its V row (a node holds
+ * all keys that reached it). Decisions are those of exact fp64 arithmetic
+ * (distances summed in index order). counts/vsum are zeroed by the call.
+ *
+ * avq_attention_deep (paper §4.3 carried down): per query row one shift (the
+ * largest level-0 logit of a non-empty node) and level-0 attention
+ * A = exp(S - m), Zbar = sum A n, Xbar = sum A vsum; then for l = 0 .. L-2
+ * the candidates (level 0: the M0 level-0 nodes; deeper: the children of
+ * the nodes expanded at l - 1, in rank order) get the importance
+ * sum_{i in tile} A_ic n_c / Zbar_i, with the Zbar so far; the P[l] largest
+ * (ties to the lower row id) are expanded, and every child g of an expanded
+ * node f adds (A_g - A_f) [vsum_g, n_g] to Xbar and Zbar. O = Xbar / Zbar.
+ * P: host array of L-1 budgets, 0 <= P[l] <= (number of candidates at l) and
+ * P[l] * C <= 128. selected: [B, H, ceil(N/tile), sum_l P[l]] int32, per
+ * tile level 0's expanded row ids by rank, then level 1's, ...
+ *
+ * Supported: 2 <= L <= 4, 1 <= M0 <= 128, C >= 1, d in {64, 128}, fp32 or
+ * bf16, tile in {64, 128}. Both calls run on CUDA cores (fp64 distances;
+ * fp32 attention). The attention workspace (fp32 value means and the status
+ * word) is avq_attention_deep_workspace_bytes(s, L) bytes, 256-byte
+ * aligned. Errors: AVQ_EINVAL (arguments), AVQ_EUNSUPPORTED (sizes),
+ * AVQ_EWORKSPACE, AVQ_ECUDA. Neither call synchronises.
+ */
+int avq_precompute_deep(const avq_shape* s, int L, const void* K, const void* V, const void* codebook,
+                        int32_t* assign, int32_t* counts, float* vsum, void* stream);
+size_t avq_attention_deep_workspace_bytes(const avq_shape* s, int L);
+int avq_attention_deep(const avq_shape* s, int L, const int32_t* P, const void* Q, const void* codebook,
+                       const int32_t* counts, const float* vsum, int tile, float scale, void* O,
+                       int32_t* selected, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Blocking: waits for `stream`, then reads the status word that kernels of
  * earlier calls using `workspace` left there (AVQ_OK; AVQ_ETIMEOUT when a
  * bounded device-side wait ran out; AVQ_ERANGE, see above) and clears it.

@@ -137,3 +137,31 @@ def test_tensor_api_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 8, 64)
     with pytest.raises(ValueError):
         bd.precompute(x, x, torch.zeros(1, 80, 64), 16, 4)
+
+
+def test_deep_argument_errors(L):
+    """Depth-L calls: depth, budgets and workspace are checked on the host."""
+    s = shape(M0=16, C=4)
+    ws = bd.avq_attention_deep_workspace_bytes(s, 3)
+    assert ws == 256 + ((1 * 2 * 16 * (1 + 4 + 16) * 64 * 4 + 255) // 256) * 256   # status + fp32 means
+    assert bd.avq_attention_deep_workspace_bytes(s, 1) == 0
+    assert bd.avq_attention_deep_workspace_bytes(s, 5) == 0
+
+    def att(P=(4, 8), Lv=3, tile=128, wsb=None, **kw):
+        a = dict(Q=FAKE, cb=FAKE, c=FAKE, v=FAKE, O=FAKE, sel=FAKE, w=FAKE)
+        a.update(kw)
+        return bd.avq_attention_deep(s, Lv, P, a["Q"], a["cb"], a["c"], a["v"], tile, 0.125, a["O"], a["sel"],
+                                     a["w"], ws if wsb is None else wsb, stream=0)
+
+    assert att(Lv=1, P=()) == -1
+    assert att(Lv=5, P=(1, 1, 1, 1)) == -1
+    assert att(P=(17, 8)) == -1        # more than the 16 level-0 nodes
+    assert att(P=(4, 17)) == -1        # more than the 4 * 4 level-1 candidates
+    assert att(P=(4, 33)) == -1        # 33 * 4 > 128 slots
+    assert att(P=(-1, 0)) == -1
+    assert att(tile=32) == -1
+    assert att(sel=0) == -1
+    assert att(wsb=0) == -5
+    assert bd.avq_precompute_deep(s, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0) == -1
+    assert bd.avq_precompute_deep(shape(M0=129, C=2), 3, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0) == -2
+    assert bd.avq_precompute_deep(s, 3, FAKE, 0, FAKE, FAKE, FAKE, FAKE, stream=0) == -1
