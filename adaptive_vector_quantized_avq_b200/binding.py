@@ -28,7 +28,7 @@ EXPORTS = ("avq_precompute_workspace_bytes", "avq_precompute", "avq_attention_wo
            "avq_attention", "avq_device_status", "avq_status_string", "avq_version",
            "avq_kernel_launches", "avq_attention_noalloc", "avq_commitment", "avq_gilbert_order",
            "avq_gather_rows", "avq_capture_workspace_bytes", "avq_capture", "avq_precompute_deep",
-           "avq_attention_deep_workspace_bytes", "avq_attention_deep")
+           "avq_attention_deep_workspace_bytes", "avq_attention_deep", "avq_test_fail_next_wait")
 
 
 class AVQError(RuntimeError):
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
         L.avq_attention_deep.argtypes = [shp, i32, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp, vp, sz,
                                          vp]
         L.avq_attention_deep.restype = i32
+        L.avq_test_fail_next_wait.argtypes = []
+        L.avq_test_fail_next_wait.restype = i32
         L.avq_kernel_launches.argtypes = []
         L.avq_kernel_launches.restype = ctypes.c_uint64
         _LIB = L
@@ -207,6 +209,10 @@ def avq_attention_deep(shape, L, P, Q, codebook, counts, vsum, tile, scale, O, s
     return lib().avq_attention_deep(ctypes.byref(shape), L, ctypes.cast(Pa, ctypes.c_void_p), _ptr(Q),
                                     _ptr(codebook), _ptr(counts), _ptr(vsum), tile, float(scale), _ptr(O),
                                     _ptr(selected), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def avq_test_fail_next_wait() -> int:
+    return lib().avq_test_fail_next_wait()
 
 
 def avq_device_status(workspace, stream=None) -> int:

@@ -85,7 +85,7 @@ const char* avq_status_string(int st) {
         case AVQ_ECUDA: return "AVQ_ECUDA: a CUDA call failed";
         case AVQ_ETIMEOUT: return "AVQ_ETIMEOUT: a bounded device-side wait ran out";
         case AVQ_EWORKSPACE: return "AVQ_EWORKSPACE: workspace missing or too small";
-        case AVQ_ERANGE: return "AVQ_ERANGE: a count-weighted child logit exceeded its query's shift by more than 60";
+        case AVQ_ERANGE: return "AVQ_ERANGE: a weight out of range (reserved)";
         default: return "unknown avq status";
     }
 }

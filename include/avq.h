@@ -57,7 +57,7 @@ typedef enum { AVQ_F32 = 0, AVQ_BF16 = 1 } avq_dtype;
  * a tree: 1 <= M0 <= 128, 1 <= C <= 16;
  * a flat codebook (C == 0, M0 codewords and no children; paper §3.2 VQ
  * attention): 1 <= M0 <= 512, bf16 only; avq_attention then takes P == 0
- * and d == 64 with tile 128 (other flat cases return AVQ_EUNSUPPORTED). */
+ * with tile 128 (other flat cases return AVQ_EUNSUPPORTED). */
 typedef struct {
     int32_t B, H, N, d;
     int32_t M0, C;
@@ -71,11 +71,7 @@ typedef enum {
     AVQ_ECUDA = -3,         /* a CUDA launch or runtime call failed */
     AVQ_ETIMEOUT = -4,      /* a bounded device-side wait ran out (reported by avq_device_status) */
     AVQ_EWORKSPACE = -5,    /* workspace missing or smaller than the *_workspace_bytes() answer */
-    AVQ_ERANGE = -6         /* (device status, bf16 tensor-core kernel) for some query, a
-                               non-empty child's scaled logit plus log n_c exceeded the common
-                               shift of that query's weights (the largest non-empty parent logit
-                               plus log n_p) by more than 60 (natural-log units): its weights may
-                               overflow fp32, and O is then not meaningful */
+    AVQ_ERANGE = -6         /* reserved (no current kernel reports it): a weight out of range */
 } avq_status;
 
 /*
@@ -171,7 +167,7 @@ int avq_attention(const avq_shape* s, const void* Q, const void* codebook,
  *   contents; calls whose work overlaps on the GPU (different streams or host
  *   threads) race on it and must be serialised by the caller.
  * - device_status (device pointer to one int32, may be NULL) receives this
- *   call's device status word (AVQ_OK, AVQ_ETIMEOUT or AVQ_ERANGE), written
+ *   call's device status word (AVQ_OK or AVQ_ETIMEOUT), written
  *   on `stream`.
  * - Allocates nothing: no cudaMalloc/cudaFree and no allocating library call.
  */
@@ -301,11 +297,23 @@ int avq_attention_deep(const avq_shape* s, int L, const int32_t* P, const void* 
 /*
  * Blocking: waits for `stream`, then reads the status word that kernels of
  * earlier calls using `workspace` left there (AVQ_OK; AVQ_ETIMEOUT when a
- * bounded device-side wait ran out; AVQ_ERANGE, see above) and clears it.
+ * bounded device-side wait ran out) and clears it.
  * Returns AVQ_ECUDA if the stream reports an error. A workspace must be
  * zero-filled before its first use.
  */
 int avq_device_status(void* workspace, void* stream);
+
+/*
+ * Test hook for the failure path (no counterpart in the paper). The next
+ * avq_attention call that runs the bf16 tensor-core tree kernel behaves as if
+ * one of its bounded device-side waits had run out: its first wait on the
+ * compute threads' first hand-over gets a limit of zero. Every CTA then stops
+ * at once: the loads and contractions it has in flight complete, its tensor
+ * memory is freed, and the call reports AVQ_ETIMEOUT through
+ * avq_device_status (its outputs are not meaningful). Later calls are
+ * unaffected. Returns AVQ_OK. Process-wide, consumed by one launch.
+ */
+int avq_test_fail_next_wait(void);
 
 /* Human-readable name of a status code (static string). */
 const char* avq_status_string(int status);

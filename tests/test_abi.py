@@ -62,7 +62,8 @@ def test_workspace_sizes(L):
     assert bd.avq_precompute_workspace_bytes(flat) >= 256
     assert bd.avq_attention_workspace_bytes(flat, 0, 128) >= 256 + 1 * 2 * 512 * 64 * 2
     assert bd.avq_attention_workspace_bytes(flat, 2, 128) == 0   # nothing to select
-    assert bd.avq_attention_workspace_bytes(shape(C=0, M0=512, d=128), 0, 128) == 0   # flat attention: d = 64
+    assert bd.avq_attention_workspace_bytes(shape(C=0, M0=512, d=128), 0, 128) >= 256 + 2 * 512 * 128 * 2
+    assert bd.avq_attention_workspace_bytes(shape(C=0, M0=512, d=128), 0, 64) == 0    # flat: tile 128 only
 
 
 FAKE = 1 << 40   # 256-byte aligned, never dereferenced: validation fails first
@@ -119,8 +120,8 @@ def test_flat_codebook_argument_rules(L):
     ws = bd.avq_attention_workspace_bytes(flat, 0, 128)
     assert bd.avq_attention(flat, FAKE, FAKE, FAKE, FAKE, 2, 128, 0.125, FAKE, FAKE, FAKE, ws,
                             stream=0) == -1
-    assert bd.avq_attention(shape(C=0, M0=256, d=128), FAKE, FAKE, FAKE, FAKE, 0, 128, 0.125, FAKE,
-                            None, FAKE, ws, stream=0) == -2
+    assert bd.avq_attention(flat, FAKE, FAKE, FAKE, FAKE, 0, 64, 0.125, FAKE, None, FAKE, ws,
+                            stream=0) == -2   # flat attention takes tile 128 only
     assert bd.avq_attention_noalloc(flat, FAKE, FAKE, FAKE, FAKE, 0, 128, 0.125, FAKE, None,
                                     stream=0) == -2
 

@@ -41,11 +41,11 @@ SMALL = [
                                     seed=15, n_components=600), (0,)),
     ("flat-3", syn.small_workload(B=1, H=1, N=200, d=64, M0=3, C=0, tile=128, dtype="bf16",
                                   seed=16, n_components=3), (0,)),
-    # head dim 128: the assignment only (the flat attention kernel is head dim 64)
+    # head dim 128 (two 64-column blocks per row, 128 output columns in TMEM)
     ("flat-d128-512", syn.small_workload(B=1, H=2, N=700, d=128, M0=512, C=0, tile=128,
-                                         dtype="bf16", seed=17, n_components=600), ()),
+                                         dtype="bf16", seed=17, n_components=600), (0,)),
     ("flat-d128-200", syn.small_workload(B=2, H=1, N=257, d=128, M0=200, C=0, tile=128,
-                                         dtype="bf16", seed=18, n_components=200), ()),
+                                         dtype="bf16", seed=18, n_components=200), (0,)),
     # dispatch paths: a bf16 tree whose codebook image does not fit the
     # tensor-core precompute's shared memory runs the CUDA-core precompute
     # (d = 64 with M0 = 128, C = 16; d = 128 with M0 = 128, C = 8); C = 16 on
@@ -153,11 +153,11 @@ def test_duplicate_parents_exact_ties(lib_built, oracle):
     print(rep)
 
 
-def test_range_flag(lib_built):
-    """A non-empty child whose logit lies far above every parent logit of the
-    queries raises AVQ_ERANGE in the attention call's device status (no fault;
-    the tensor-core kernel reports it after the launch)."""
-    from adaptive_vector_quantized_avq_b200 import binding as bd
+def test_far_child_moves_the_shift(lib_built, oracle):
+    """A non-empty child whose logit lies about 127 octaves above every parent
+    logit of the queries: the row's shift moves up (the running accumulators
+    are rescaled by an exact power of two, paper §4.3) and the output and
+    selection are still the oracle's, with no overflow and no device error."""
     d, M0, C, N = 64, 16, 2, 256
     rng = np.random.default_rng(12)
     grid = 1.0 / 32
@@ -168,16 +168,42 @@ def test_range_flag(lib_built):
     cb = np.concatenate([par, ch])[None]                                # [1, Mtot, d]
     K = np.round(rng.standard_normal((1, 1, N, d)) * 0.1 / grid) * grid
     K[0, 0, 0] = 3.0                                                    # a key on the far child
-    # q . child0 = 96 against q . parent0 = 8 (scale 1): ~80 nats above the shift
+    V = rng.standard_normal((1, 1, N, d))
+    # q . child0 = 96 against q . parent0 = 8 (scale 1): ~127 octaves above the shift
     Q = np.full((1, 1, N, d), 0.5)
-    dev = "cuda"
-    t = lambda a: parity.to_device(syn.f64_to_bf16_bits(a), "bf16", dev)
-    Kt, Qt, cbt = t(K), t(Q), t(cb)
-    assign, counts, vsum = bd.precompute(Kt, Kt, cbt, M0, C)
-    torch.cuda.synchronize()
-    assert int(assign[0, 0, 0]) == M0   # the far key sits on child 0 of parent 0
-    shape = bd.make_shape(1, 1, N, d, M0, C, Qt.dtype)
-    ws = bd.workspace(bd.avq_attention_workspace_bytes(shape, M0, 128), Qt.device)
-    bd.attention(Qt, cbt, counts, vsum, M0, C, M0, 128, 1.0, ws=ws)
-    assert bd.avq_device_status(ws) == -6
-    assert bd.avq_device_status(ws) == 0   # reading the status clears it
+    wl = syn.small_workload(B=1, H=1, N=N, d=d, M0=M0, C=C, tile=128, dtype="bf16", P=(M0, 3),
+                            scale=1.0)
+    store = lambda a: syn.f64_to_bf16_bits(a)
+    inp = syn.Inputs(wl, store(K), store(V), store(Q), store(cb))
+    gpu = parity.run_gpu(wl, inp, wl.P)   # asserts a clean device status
+    assert int(gpu["assign"][0, 0, 0]) == M0   # the far key sits on child 0 of parent 0
+    ora = oracle.precompute(inp.f64("K"), inp.f64("V"), inp.f64("codebook"), M0, C)
+    parity.check_precompute(wl, inp, gpu, ora, oracle)
+    for P in wl.P:
+        O, sel = gpu["att"][P]
+        rep = parity.check_attention(wl, inp, P, O, sel, ora["counts"], ora["vsum"], oracle)
+        print(P, dict(rep))
+
+
+def test_timeout_status_and_recovery(lib_built, oracle):
+    """The failure path of a bounded wait, without a GPU fault: the test hook
+    gives the attention kernel's first hand-over wait a limit of zero. The call
+    reports AVQ_ETIMEOUT through the device status (every CTA stopped, drained
+    its loads and contractions and freed its tensor memory), and the next call
+    on the same context is correct and clean."""
+    from adaptive_vector_quantized_avq_b200 import binding as bd
+    wl = syn.small_workload(B=1, H=2, N=700, d=64, M0=32, C=4, tile=128, dtype="bf16", seed=24,
+                            n_components=40, P=(6,))
+    inp = syn.generate(wl)
+    K, V, Q, cb = (parity.to_device(getattr(inp, n), wl.dtype) for n in ("K", "V", "Q", "codebook"))
+    _, counts, vsum = bd.precompute(K, V, cb, wl.M0, wl.C)
+    shape = bd.make_shape(wl.B, wl.H, wl.N, wl.d, wl.M0, wl.C, Q.dtype)
+    ws = bd.workspace(bd.avq_attention_workspace_bytes(shape, 6, 128), Q.device)
+    assert bd.avq_test_fail_next_wait() == 0
+    bd.attention(Q, cb, counts, vsum, wl.M0, wl.C, 6, 128, wl.softmax_scale, ws=ws)
+    assert bd.avq_device_status(ws) == -4          # AVQ_ETIMEOUT
+    O, sel = bd.attention(Q, cb, counts, vsum, wl.M0, wl.C, 6, 128, wl.softmax_scale, ws=ws)
+    assert bd.avq_device_status(ws) == 0
+    ora = oracle.precompute(inp.f64("K"), inp.f64("V"), inp.f64("codebook"), wl.M0, wl.C)
+    parity.check_attention(wl, inp, 6, parity.from_device(O), sel.cpu().numpy(), ora["counts"], ora["vsum"],
+                           oracle)
