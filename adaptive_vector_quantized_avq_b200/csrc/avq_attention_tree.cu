@@ -238,9 +238,9 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     float* sX = sLc + 128;                   // [2][128] row exchange: shift
     float* sZ = sX + 256;                    // [2][128] row exchange: Zbar, then the denominator
     float* sT = sZ + 256;                    // [2][128] row exchange: largest child exponent
-    unsigned long long* sKey = reinterpret_cast<unsigned long long*>(sT + 256);   // [128] rank keys
-    int* sRank = reinterpret_cast<int*>(sKey + 128);           // [2][128] partial ranks
-    int* sSel = sRank + 256;                                   // [128] selected parents by rank
+    uint32_t* sKey = reinterpret_cast<uint32_t*>(sT + 256);   // [128] importance bits
+    int* sRank = reinterpret_cast<int*>(sKey + 128);           // [2][2][128] partial ranks, partial equal counts
+    int* sSel = sRank + 512;                                   // [128] selected parents by rank
     uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + 128);
     uint64_t* bQ = bars;                     // [2] Q stage landed
     uint64_t* bHead = bars + 2;              // head tables landed
@@ -584,29 +584,44 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                 tc_fence_before();   // the reads of e' precede MMA2 (issued after later hand-overs)
                 if (wg_sync_or(!ok)) { failed = true; break; }
 
-                // ---- top-P by ranks over unique 64-bit keys: the bit pattern of the
-                // importance (w >= 0 orders like its bits), then the complement of the
-                // index (ties to the lower index); the two threads of a row count the
-                // larger keys among half of the parents each
+                // ---- top-P by ranks: the key of a parent is the bit pattern of its
+                // importance (w >= 0 orders like its bits); its rank the number of
+                // larger keys, ties to the lower index. The two threads of a row count
+                // over half of the parents each, with 32-bit compares; when a selected
+                // candidate's key is shared, every rank is taken again over 64-bit keys
+                // (bits, then the complement of the index), which are unique.
                 if (store_thread) bulk_wait_read_all();   // the previous O store has read the staging
                 {
                     const float w = (sPart[r] + sPart[128 + r]) + (sPart[256 + r] + sPart[384 + r]);
-                    const unsigned long long key =
-                        ((unsigned long long)(r < p.M0 ? __float_as_uint(w) : 0u) << 32) | (uint32_t)(0xFFFFFFFFu - r);
-                    if (hf == 0) sKey[r] = key;
+                    const uint32_t kr = r < p.M0 ? __float_as_uint(w) : 0u;
+                    if (hf == 0) sKey[r] = kr;
                     wg_sync();
-                    int gt0 = 0, gt1 = 0;
+                    int gt0 = 0, gt1 = 0, eq0 = 0, eq1 = 0;
                     const int qe = min(64 * hf + 64, p.M0p);
 #pragma unroll 4
-                    for (int qq = 64 * hf; qq < qe; qq += 4) {
-                        const ulonglong2 k0 = *reinterpret_cast<const ulonglong2*>(sKey + qq);
-                        const ulonglong2 k1 = *reinterpret_cast<const ulonglong2*>(sKey + qq + 2);
-                        gt0 += (k0.x > key) + (k0.y > key);
-                        gt1 += (k1.x > key) + (k1.y > key);
+                    for (int qq = 64 * hf; qq < qe; qq += 8) {
+                        const uint4 k0 = *reinterpret_cast<const uint4*>(sKey + qq);
+                        const uint4 k1 = *reinterpret_cast<const uint4*>(sKey + qq + 4);
+                        gt0 += (k0.x > kr) + (k0.y > kr) + (k0.z > kr) + (k0.w > kr);
+                        gt1 += (k1.x > kr) + (k1.y > kr) + (k1.z > kr) + (k1.w > kr);
+                        eq0 += (k0.x == kr) + (k0.y == kr) + (k0.z == kr) + (k0.w == kr);
+                        eq1 += (k1.x == kr) + (k1.y == kr) + (k1.z == kr) + (k1.w == kr);
                     }
                     sRank[hf * 128 + r] = gt0 + gt1;
+                    sRank[256 + hf * 128 + r] = eq0 + eq1;
                     pair_sync(q);
-                    const int rank = sRank[r] + sRank[128 + r];
+                    int rank = sRank[r] + sRank[128 + r];
+                    const bool tie =
+                        wg_sync_or(hf == 0 && r < p.M0 && rank < p.P && sRank[256 + r] + sRank[384 + r] > 1);
+                    if (tie) {
+                        const unsigned long long key = ((unsigned long long)kr << 32) | (uint32_t)(0xFFFFFFFFu - r);
+                        int rk = 0;
+                        for (int qq = 64 * hf; qq < qe; ++qq)
+                            rk += (((unsigned long long)sKey[qq] << 32) | (uint32_t)(0xFFFFFFFFu - qq)) > key;
+                        sRank[hf * 128 + r] = rk;   // (every thread read the partial ranks before the barrier)
+                        pair_sync(q);
+                        rank = sRank[r] + sRank[128 + r];
+                    }
                     if (hf == 0 && r < p.M0 && rank < p.P) {
                         sSel[rank] = r;
                         p.selected[((size_t)bh * p.ntiles + t) * p.P + rank] = r;
@@ -872,9 +887,9 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 }
 
 size_t tree_smem(int D, int M0, int C) {
-    // 1 KB alignment, six [128 x D] images, 20 x 128 words of tables, 12 mbarriers,
+    // 1 KB alignment, six [128 x D] images, 22 x 128 words of tables, 12 mbarriers,
     // 4 words, the child counts of one (b,h)
-    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 20 + 12 * 8 + 16 + (size_t)M0 * C * 4;
+    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 22 + 12 * 8 + 16 + (size_t)M0 * C * 4;
 }
 
 template <int D, int C>

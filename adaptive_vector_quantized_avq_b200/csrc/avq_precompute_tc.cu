@@ -427,8 +427,19 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             mph ^= 1;
             tc_fence_after();
 
-            // ---- a1, pass 1: the smallest v_p = ||C_p||^2 - 2 S_p
-            float m = INFINITY;
+            // this key's V row is read after the children: start bringing it to L2 now
+            if (valid) {
+                const char* vrow = reinterpret_cast<const char*>(p.V + ((size_t)bh * p.N + (size_t)t * kTile + lt) * D);
+#pragma unroll
+                for (int o = 0; o < D * 2; o += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(vrow + o));
+            }
+
+            // ---- a1: v_p = ||C_p||^2 - 2 S_p in one pass over TMEM, keeping the
+            // smallest (and its index) and the second smallest (two trackers, even
+            // and odd columns, merged after). A parent is certainly the nearest
+            // when the runner-up lies above the error band of the smallest.
+            float m1a = INFINITY, m2a = INFINITY, m1b = INFINITY, m2b = INFINITY;
+            int i1a = 0, i1b = 0;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 if (16 * c < p.M0p) {
@@ -439,11 +450,26 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 #pragma unroll
                     for (int q = 0; q < 16; q += 4) {
                         const float4 cn4 = *reinterpret_cast<const float4*>(sCn + 16 * c + q);
-                        m = fmin3(m, fmaf(-2.f, v16[q], cn4.x), fmaf(-2.f, v16[q + 1], cn4.y));
-                        m = fmin3(m, fmaf(-2.f, v16[q + 2], cn4.z), fmaf(-2.f, v16[q + 3], cn4.w));
+                        const float cnq[4] = {cn4.x, cn4.y, cn4.z, cn4.w};
+#pragma unroll
+                        for (int u = 0; u < 4; u += 2) {
+                            const float va = fmaf(-2.f, v16[q + u], cnq[u]);
+                            const float vb = fmaf(-2.f, v16[q + u + 1], cnq[u + 1]);
+                            const bool la = va < m1a, lb = vb < m1b;
+                            m2a = la ? m1a : fminf(m2a, va);
+                            m2b = lb ? m1b : fminf(m2b, vb);
+                            i1a = la ? 16 * c + q + u : i1a;
+                            i1b = lb ? 16 * c + q + u + 1 : i1b;
+                            m1a = la ? va : m1a;
+                            m1b = lb ? vb : m1b;
+                        }
                     }
                 }
             }
+            const bool use_a = m1a < m1b || (m1a == m1b && i1a < i1b);
+            const float m = use_a ? m1a : m1b;
+            const int im = use_a ? i1a : i1b;
+            const float m2 = fminf(fminf(m2a, m2b), use_a ? m1b : m1a);
 
             // ||k||^2 straight from the bf16 key row (the row itself is
             // loaded again once the parent is known, to keep registers free)
@@ -461,33 +487,14 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                 kn = __fadd_rn(kn0, kn1);
             }
 
-            // ---- a1, pass 2: the parents within the error band of the
-            // smallest (count in the low byte, their index sum above it); a
-            // single one is certainly the nearest
+            // the parents within the error band of the smallest: a single one (the
+            // runner-up above the band) is certainly the nearest; otherwise the key
+            // is listed for the fp64 decision (parent 0 stands in until then)
             const float E = c_exp * (kn + cnmax);
             const float thr = __fadd_ru(m, 2.f * E);
-            int acc = 0;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                if (16 * c < p.M0p) {
-                    float v16[16];
-                    tmem_ld16f(trow + 16 * c, v16);
-                    tmem_wait_ld();
-                    tmem_touch16f(v16);
-#pragma unroll
-                    for (int q = 0; q < 16; q += 4) {
-                        const float4 cn4 = *reinterpret_cast<const float4*>(sCn + 16 * c + q);
-                        const float cnq[4] = {cn4.x, cn4.y, cn4.z, cn4.w};
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            if (fmaf(-2.f, v16[q + u], cnq[u]) <= thr) acc += ((16 * c + q + u) << 8) + 1;
-                    }
-                }
-            }
-            // more than one parent in the band: decided later in fp64 (the key
-            // is listed; parent 0 stands in until then)
-            int bp = (acc & 255) == 1 ? (acc >> 8) : 0;
-            bool listed = valid && (acc & 255) != 1;
+            const bool single = m2 > thr;
+            int bp = single ? im : 0;
+            bool listed = valid && !single;
             n_pre += listed;
             // key row (packed bf16) -> registers
             uint4 kw[D / 8];
@@ -532,7 +539,7 @@ precompute_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             if (listed) {
                 const int slot = atomicAdd(sFix, 1);
                 const long long kidx = (long long)bh * p.N + (long long)t * kTile + lt;
-                p.fix_list[(size_t)g0 * kTile + slot] = (acc & 255) == 1 ? kidx | ((long long)(bp + 1) << 40) : kidx;
+                p.fix_list[(size_t)g0 * kTile + slot] = single ? kidx | ((long long)(bp + 1) << 40) : kidx;
             }
 
             // ---- a3: outputs. Counts and value sums go to the leaf only (the
