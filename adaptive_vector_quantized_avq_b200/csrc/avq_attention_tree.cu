@@ -32,10 +32,10 @@
 //      importance), bf16 W_p -> TMEM; MMA3p O = W_p x mean_par.
 //   2. Importance w_p = sum_rows e'_p / Zbar, from TMEM in the 16x256b
 //      layout (each thread holds four rows), a three-level butterfly and a
-//      four-warp sum in shared memory; top-P by ranks over 32-bit keys (the
-//      bit patterns of w >= 0), re-ranked over 64-bit keys (bits, then the
-//      complement of the index: ties to the lower index) when leading keys
-//      tie.
+//      four-warp sum in shared memory; top-P over 64-bit values (the bit
+//      pattern of w >= 0 above the complement of the index: ties to the lower
+//      index), each of four warps sorting 32 of them, a value's rank found
+//      by binary searches in the other warps' lists.
 //   3. Per chunk of <= 128 selected child slots: the compute threads gather
 //      the children's codewords and value means (cp.async), the producer
 //      issues MMA2 S_c; the child weight (A_c - A_p) n_c = 2^(x_c - m) -
@@ -212,6 +212,51 @@ __device__ __forceinline__ void butterfly_level(float* v, bool up, int mask) {
     }
 }
 
+// The tile's top-P parents, in rank order, into sel (shared) and out (global),
+// by four warps (quarter q holds parents 32q .. 32q + 31, one per lane). Each
+// parent's value is the bit pattern of its importance w >= 0 (which orders like
+// w) above the complement of its index, so that ties go to the lower index;
+// parents past M0 sort last. Each warp sorts its 32 values (bitonic, 15
+// shuffle steps) and publishes them; a value's rank is its place in its own
+// list plus, for each other list, the number of larger values there (a binary
+// search). list: 128 64-bit words of shared memory.
+__device__ __forceinline__ void select_top_p4(const float* part, unsigned long long* list, int* sel, int32_t* out,
+                                              int M0, int P, int q, int lane) {
+    const int par = 32 * q + lane;
+    const float w = (part[par] + part[128 + par]) + (part[256 + par] + part[384 + par]);
+    const uint32_t key = par < M0 ? __float_as_uint(w) : 0u;
+    unsigned long long v = ((unsigned long long)key << 32) | (uint32_t)(0xFFFFFFFFu - par);
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
+            v = (v > o) == keep_max ? v : o;
+        }
+    }
+    list[32 * q + lane] = v;
+    asm volatile("bar.sync 6, 128;" ::: "memory");
+    if (lane < P) {
+        int rank = lane;
+#pragma unroll
+        for (int d = 1; d < 4; ++d) {
+            const unsigned long long* L = list + 32 * ((q + d) & 3);
+            int c = 0;   // number of values in L above v (L is descending)
+#pragma unroll
+            for (int step = 16; step > 0; step >>= 1)
+                if (L[c + step - 1] > v) c += step;
+            c += L[c] > v;   // (c <= 31 here)
+            rank += c;
+        }
+        if (rank < P) {
+            const int pr = (int)(0xFFFFFFFFu - (uint32_t)v);
+            sel[rank] = pr;
+            out[rank] = pr;
+        }
+    }
+}
+
 template <int D, int C, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB)
 attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
@@ -235,12 +280,10 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     float* sPart = sRz + 128;                // [4][128] importance partials per quarter
     float* sNc = sPart + 512;                // [128] child counts of the chunk's slots
     float* sLc = sNc + 128;                  // [128] their log2 (-inf if empty)
-    float* sX = sLc + 128;                   // [2][128] row exchange: shift
+    float* sX = sLc + 128;                   // [2][128] row exchange: shift; the selection's sorted lists
     float* sZ = sX + 256;                    // [2][128] row exchange: Zbar, then the denominator
     float* sT = sZ + 256;                    // [2][128] row exchange: largest child exponent
-    uint32_t* sKey = reinterpret_cast<uint32_t*>(sT + 256);   // [128] importance bits
-    int* sRank = reinterpret_cast<int*>(sKey + 128);           // [2][2][128] partial ranks, partial equal counts
-    int* sSel = sRank + 512;                                   // [128] selected parents by rank
+    int* sSel = reinterpret_cast<int*>(sT + 256);              // [128] selected parents by rank
     uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + 128);
     uint64_t* bQ = bars;                     // [2] Q stage landed
     uint64_t* bHead = bars + 2;              // head tables landed
@@ -584,60 +627,31 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                 tc_fence_before();   // the reads of e' precede MMA2 (issued after later hand-overs)
                 if (wg_sync_or(!ok)) { failed = true; break; }
 
-                // ---- top-P by ranks: the key of a parent is the bit pattern of its
-                // importance (w >= 0 orders like its bits); its rank the number of
-                // larger keys, ties to the lower index. The two threads of a row count
-                // over half of the parents each, with 32-bit compares; when a selected
-                // candidate's key is shared, every rank is taken again over 64-bit keys
-                // (bits, then the complement of the index), which are unique.
+                // ---- top-P: the parents ordered by (importance, then the lower
+                // index), the first P selected in rank order (select_top_p4)
+                if (hf == 0)
+                    select_top_p4(sPart, reinterpret_cast<unsigned long long*>(sX), sSel,
+                                  p.selected + ((size_t)bh * p.ntiles + t) * p.P, p.M0, p.P, q, lane);
                 if (store_thread) bulk_wait_read_all();   // the previous O store has read the staging
+                wg_sync();   // the selection is in sSel
                 {
-                    const float w = (sPart[r] + sPart[128 + r]) + (sPart[256 + r] + sPart[384 + r]);
-                    const uint32_t kr = r < p.M0 ? __float_as_uint(w) : 0u;
-                    if (hf == 0) sKey[r] = kr;
-                    wg_sync();
-                    int gt0 = 0, gt1 = 0, eq0 = 0, eq1 = 0;
-                    const int qe = min(64 * hf + 64, p.M0p);
-#pragma unroll 4
-                    for (int qq = 64 * hf; qq < qe; qq += 8) {
-                        const uint4 k0 = *reinterpret_cast<const uint4*>(sKey + qq);
-                        const uint4 k1 = *reinterpret_cast<const uint4*>(sKey + qq + 4);
-                        gt0 += (k0.x > kr) + (k0.y > kr) + (k0.z > kr) + (k0.w > kr);
-                        gt1 += (k1.x > kr) + (k1.y > kr) + (k1.z > kr) + (k1.w > kr);
-                        eq0 += (k0.x == kr) + (k0.y == kr) + (k0.z == kr) + (k0.w == kr);
-                        eq1 += (k1.x == kr) + (k1.y == kr) + (k1.z == kr) + (k1.w == kr);
-                    }
-                    sRank[hf * 128 + r] = gt0 + gt1;
-                    sRank[256 + hf * 128 + r] = eq0 + eq1;
-                    pair_sync(q);
-                    int rank = sRank[r] + sRank[128 + r];
-                    const bool tie =
-                        wg_sync_or(hf == 0 && r < p.M0 && rank < p.P && sRank[256 + r] + sRank[384 + r] > 1);
-                    if (tie) {
-                        const unsigned long long key = ((unsigned long long)kr << 32) | (uint32_t)(0xFFFFFFFFu - r);
-                        int rk = 0;
-                        for (int qq = 64 * hf; qq < qe; ++qq)
-                            rk += (((unsigned long long)sKey[qq] << 32) | (uint32_t)(0xFFFFFFFFu - qq)) > key;
-                        sRank[hf * 128 + r] = rk;   // (every thread read the partial ranks before the barrier)
-                        pair_sync(q);
-                        rank = sRank[r] + sRank[128 + r];
-                    }
-                    if (hf == 0 && r < p.M0 && rank < p.P) {
-                        sSel[rank] = r;
-                        p.selected[((size_t)bh * p.ntiles + t) * p.P + rank] = r;
-                        if (tma_gather) {   // this parent's children: slot tables and one TMA load per image
-#pragma unroll
-                            for (int c = 0; c < C; ++c) {
-                                const float nc = sCnt[r * C + c];
-                                sNc[rank * C + c] = nc;
-                                sLc[rank * C + c] = nc > 0.f ? __log2f(nc) : -INFINITY;
-                            }
+                    if (tma_gather) {   // each selected parent's children: one TMA load per image
+                        // (slot s from thread 32 (s % 8) + s / 8: the loads leave from all
+                        // eight warps, not one warp's lanes in turn)
+                        const int gslot = (ct & 31) * 8 + (ct >> 5);
+                        if (gslot < p.P) {
+                            const int par = min(max(sSel[gslot], 0), p.M0 - 1);
                             mbar_arrive_expect_tx(bGatT, 2u * KH * (uint32_t)C * 128u);
 #pragma unroll
                             for (int kh = 0; kh < KH; ++kh) {
-                                tma_load_3d(sCC + kh * kRegion + rank * C * 128, &tmCBc, bGatT, kh * 64, p.M0 + r * C, h);
-                                tma_load_3d(sMC + kh * kRegion + rank * C * 128, &tmMNc, bGatT, kh * 64, p.M0 + r * C, bh);
+                                tma_load_3d(sCC + kh * kRegion + gslot * C * 128, &tmCBc, bGatT, kh * 64, p.M0 + par * C, h);
+                                tma_load_3d(sMC + kh * kRegion + gslot * C * 128, &tmMNc, bGatT, kh * 64, p.M0 + par * C, bh);
                             }
+                        }
+                        if (ct < PC) {   // slot tables: the child's count and its log2
+                            const float nc = sCnt[min(max(sSel[ct / C], 0), p.M0 - 1) * C + ct % C];
+                            sNc[ct] = nc;
+                            sLc[ct] = nc > 0.f ? __log2f(nc) : -INFINITY;
                         }
                     }
                     if (tma_gather && ct == 255) {   // the chunk's padding slots: zero rows, empty entries
@@ -699,33 +713,75 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                     sph ^= 1;
                     tc_fence_after();
                     wg_sync();           // the slot tables and the selection are complete
-                    // this thread's 16-slot blocks 2i + hf; first the row's largest
-                    // exponent t = sl2 S_c + log2 n_c - m (both threads), then the weights
+                    // child weights (A_c - A_p) n_c = 2^t - A_p n_c with t = sl2 S_c +
+                    // log2 n_c - m, over this thread's 16-slot blocks 2i + hf, rounded to
+                    // bf16 once; the denominator from the same rounded values. They are
+                    // held until both threads of the row have read their S_c, then
+                    // written as W_c over the S_c columns. When the row's largest t is
+                    // above 64 the shift moves up by whole octaves: O, W_p and the
+                    // denominator are scaled by 2^-k (exact) and the weights taken again
+                    // (paper §4.3: the running accumulators follow the maximum).
                     const int nb = (N2 / 16 + 1 - hf) / 2;
-                    const float2 negm0 = make_float2(-m, -m);
-                    float tmax = -INFINITY;
-                    for (int i = 0; i < nb; ++i) {
-                        const int b = 2 * i + hf;
-                        float sc[16];
-                        tmem_ld16f(trow + 16 * b, sc);
-                        tmem_wait_ld();
-                        tmem_touch16f(sc);
+                    float2 dc0, dc1;
+                    uint32_t wall[4][8];
+#pragma unroll 1
+                    for (int attempt = 0;; ++attempt) {
+                        const float2 negm = make_float2(-m, -m);
+                        float tmax = -INFINITY;
+                        dc0 = make_float2(0.f, 0.f);
+                        dc1 = make_float2(0.f, 0.f);
 #pragma unroll
-                        for (int kk = 0; kk < 16; kk += 4) {
-                            const float4 lc = *reinterpret_cast<const float4*>(sLc + 16 * b + kk);
-                            const float2 t0 = ffma2(make_float2(sc[kk], sc[kk + 1]), sl2v, fadd2(make_float2(lc.x, lc.y), negm0));
-                            const float2 t1 = ffma2(make_float2(sc[kk + 2], sc[kk + 3]), sl2v, fadd2(make_float2(lc.z, lc.w), negm0));
-                            tmax = fmax3(tmax, fmax3(t0.x, t0.y, t1.x), t1.y);
+                        for (int i = 0; i < 4; ++i) {
+                            if (i >= nb) break;
+                            const int b = 2 * i + hf;
+                            constexpr int PB = C >= 16 ? 1 : 16 / C;   // parents behind a 16-slot block
+                            float sc[16];
+                            float nap[PB];
+                            {
+                                int pid[PB];
+                                uint32_t wr[PB];
+                                tmem_ld16f(trow + 16 * b, sc);
+#pragma unroll
+                                for (int j = 0; j < PB; ++j) {
+                                    pid[j] = min(max(sSel[min((cs + 16 * b) / C + j, p.P - 1)], 0), p.M0 - 1);
+                                    tmem_ld1(trow + p.colWp + (pid[j] >> 1), wr[j]);
+                                }
+                                tmem_wait_ld();
+                                tmem_touch16f(sc);
+#pragma unroll
+                                for (int j = 0; j < PB; ++j) {
+                                    tmem_touch1(wr[j]);
+                                    nap[j] = -((pid[j] & 1) ? bf16_hi(wr[j]) : bf16_lo(wr[j])) * sInvN[pid[j]];
+                                }
+                            }
+#pragma unroll
+                            for (int kk = 0; kk < 16; kk += 4) {
+                                const float4 lc = *reinterpret_cast<const float4*>(sLc + 16 * b + kk);
+                                const float4 nc = *reinterpret_cast<const float4*>(sNc + 16 * b + kk);
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int s = kk + 2 * e;
+                                    const float2 tt = ffma2(make_float2(sc[s], sc[s + 1]), sl2v,
+                                                            fadd2(e ? make_float2(lc.z, lc.w) : make_float2(lc.x, lc.y), negm));
+                                    tmax = fmax3(tmax, tt.x, tt.y);
+                                    const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));
+                                    const float2 wc = ffma2(make_float2(nap[s / C < PB ? s / C : 0], nap[(s + 1) / C < PB ? (s + 1) / C : 0]),
+                                                            e ? make_float2(nc.z, nc.w) : make_float2(nc.x, nc.y), ev);
+                                    const uint32_t wb = pack_bf16x2(wc.x, wc.y);
+                                    const float2 wr2 = make_float2(bf16_lo(wb), bf16_hi(wb));
+                                    if (e) dc1 = fadd2(dc1, wr2);
+                                    else dc0 = fadd2(dc0, wr2);
+                                    wall[i][s >> 1] = wb;
+                                }
+                            }
                         }
-                    }
-                    sT[hf * 128 + r] = tmax;
-                    pair_sync(q);
-                    tmax = fmaxf(sT[r], sT[128 + r]);
-                    const bool up = tmax > kRescale;
-                    if (__any_sync(0xffffffffu, up)) {
-                        // A child far above the shift: move it up by k whole octaves and
-                        // scale O, W_p and the denominator by 2^-k (exact). The TMEM accesses
-                        // are warp-collective: rows that keep their shift take factor 1.
+                        sT[hf * 128 + r] = tmax;
+                        pair_sync(q);   // both threads' S_c and W_p reads precede any write to them
+                        tmax = fmaxf(sT[r], sT[128 + r]);
+                        const bool up = attempt == 0 && tmax > kRescale;
+                        if (!__any_sync(0xffffffffu, up)) break;
+                        // (rare) The TMEM accesses are warp-collective: rows that keep
+                        // their shift take factor 1.
                         const int kup = up ? (int)ceilf(fminf(tmax, 1.0e6f)) : 0;
                         const float f = exp2_neg_int(kup);
                         m += (float)kup;
@@ -753,62 +809,10 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                         tmem_wait_st();
                         pair_sync(q);   // the partner's blocks of W_p are scaled too
                     }
-                    // child weights (A_c - A_p) n_c = 2^t - A_p n_c, rounded to bf16 once;
-                    // the denominator from the same rounded values. They are held until
-                    // both threads of the row have read their S_c, then written as W_c
-                    // over the S_c columns.
-                    const float2 negm = make_float2(-m, -m);
-                    float2 dc0 = make_float2(0.f, 0.f), dc1 = make_float2(0.f, 0.f);
-                    uint32_t wall[4][8];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (i >= nb) break;
-                        const int b = 2 * i + hf;
-                        constexpr int PB = C >= 16 ? 1 : 16 / C;   // parents behind a 16-slot block
-                        float sc[16];
-                        float nap[PB];
-                        {
-                            int pid[PB];
-                            uint32_t wr[PB];
-                            tmem_ld16f(trow + 16 * b, sc);
-#pragma unroll
-                            for (int j = 0; j < PB; ++j) {
-                                pid[j] = min(max(sSel[min((cs + 16 * b) / C + j, p.P - 1)], 0), p.M0 - 1);
-                                tmem_ld1(trow + p.colWp + (pid[j] >> 1), wr[j]);
-                            }
-                            tmem_wait_ld();
-                            tmem_touch16f(sc);
-#pragma unroll
-                            for (int j = 0; j < PB; ++j) {
-                                tmem_touch1(wr[j]);
-                                nap[j] = -((pid[j] & 1) ? bf16_hi(wr[j]) : bf16_lo(wr[j])) * sInvN[pid[j]];
-                            }
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < 16; kk += 4) {
-                            const float4 lc = *reinterpret_cast<const float4*>(sLc + 16 * b + kk);
-                            const float4 nc = *reinterpret_cast<const float4*>(sNc + 16 * b + kk);
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int s = kk + 2 * e;
-                                const float2 tt = ffma2(make_float2(sc[s], sc[s + 1]), sl2v,
-                                                        fadd2(e ? make_float2(lc.z, lc.w) : make_float2(lc.x, lc.y), negm));
-                                const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));
-                                const float2 wc = ffma2(make_float2(nap[s / C < PB ? s / C : 0], nap[(s + 1) / C < PB ? (s + 1) / C : 0]),
-                                                        e ? make_float2(nc.z, nc.w) : make_float2(nc.x, nc.y), ev);
-                                const uint32_t wb = pack_bf16x2(wc.x, wc.y);
-                                const float2 wr2 = make_float2(bf16_lo(wb), bf16_hi(wb));
-                                if (e) dc1 = fadd2(dc1, wr2);
-                                else dc0 = fadd2(dc0, wr2);
-                                wall[i][s >> 1] = wb;
-                            }
-                        }
-                    }
                     // W_c goes over the chunk's S_c columns, except for the tile's last
                     // chunk: that one goes over W_p (no lookup needs it any more), so
                     // that the next tile's MMA1 may write the S columns while the last
                     // MMA3c still reads W_c
-                    pair_sync(q);   // both threads' S_c and W_p reads precede any W_c write
                     const uint32_t colWc = k + 1 == nchunks ? p.colWp : 0u;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -887,9 +891,9 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 }
 
 size_t tree_smem(int D, int M0, int C) {
-    // 1 KB alignment, six [128 x D] images, 22 x 128 words of tables, 12 mbarriers,
+    // 1 KB alignment, six [128 x D] images, 16 x 128 words of tables, 12 mbarriers,
     // 4 words, the child counts of one (b,h)
-    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 22 + 12 * 8 + 16 + (size_t)M0 * C * 4;
+    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 16 + 12 * 8 + 16 + (size_t)M0 * C * 4;
 }
 
 template <int D, int C>
