@@ -66,7 +66,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kTile = 128;
-constexpr int kThreads = 288;
+constexpr int kThreads = 256;
+constexpr int kBars = 8;                  // mbarriers in shared memory
 constexpr uint32_t kRegion = 128 * 128;   // one 64-column block of a 128-row bf16 image
 constexpr float kRescale = 64.f;          // largest child weight exponent (log2) before the shift moves
 
@@ -100,30 +101,9 @@ __device__ __forceinline__ uint32_t swz(int r, int j) {
     return (uint32_t)(j >> 3) * kRegion + (uint32_t)r * 128u + (uint32_t)(((j & 7) ^ (r & 7)) << 4);
 }
 
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -290,17 +270,18 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     uint64_t* bS = bars + 3;                 // MMA1 / MMA2 done (S_p, S_c ready)
     uint64_t* bO = bars + 4;                 // the tile's last contraction done
     uint64_t* bC = bars + 5;                 // a chunk's contraction done (all but the last)
-    uint64_t* bWp = bars + 6;                // (256) W_p written
-    uint64_t* bGat = bars + 7;               // (256) a chunk's children gathered (e' read)
-    uint64_t* bWc = bars + 8;                // (256) W_c written
-    uint64_t* bEpi = bars + 9;               // (256) O read
-    uint64_t* bFin = bars + 10;              // (failure only) contractions in flight done
-    uint64_t* bGatT = bars + 11;             // (P + 1, tx) the selected parents' children landed (TMA)
-    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 12);
+    uint64_t* bFin = bars + 6;               // (failure only) contractions in flight done
+    uint64_t* bGatT = bars + 7;              // (P + 1, tx) the selected parents' children landed (TMA)
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + kBars);
     volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
     float* sCnt = reinterpret_cast<float*>(sTmem + 4);        // [M0 * C] this (b,h)'s child counts
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3;                  // TMEM lane quarter of this warp
+    const int hf = warp >> 2;                // which half of the row's columns
+    const int r = 32 * q + lane;             // query row (and parent / slot index)
+    const bool leader = tid == 0;            // issues the Q and head loads and every tcgen05.mma
+    const bool store_thread = tid == 32;     // issues the O stores
     const int g0 = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
     const int g1 = (int)(((long long)(blockIdx.x + 1) * p.total_tiles) / gridDim.x);
     const int PC = p.P * C;
@@ -320,10 +301,6 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         mbar_init(bS, 1);
         mbar_init(bO, 1);
         mbar_init(bC, 1);
-        mbar_init(bWp, 256);
-        mbar_init(bGat, 256);
-        mbar_init(bWc, 256);
-        mbar_init(bEpi, 256);
         mbar_init(bFin, 1);
         mbar_init(bGatT, tma_gather ? p.P + 1 : 1);
         *sAbort = 0;
@@ -344,536 +321,508 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *sTmem;
     bool failed = false;
-    // (producer) loads issued but not yet seen complete, for the failure path
-    uint32_t q_pending = 0, qph = 0, hph = 0;
-    bool head_pending = false;
+    // (leader) loads issued but not yet seen complete, for the failure path
+    uint32_t q_pending = 0, qph = 0, hph = 0, gtph = 0;
+    bool head_pending = false, gat_pending = false;
+    const uint32_t idesc1 = idesc_bf16_f32(128, p.M0p, false);
+    const uint32_t idesc3 = idesc_bf16_f32(128, D, true);
+    // (leader) the TMA load of tile g's Q into stage `stage`
+    auto issue_q = [&](int g, int stage) {
+        const int bh = g / p.ntiles, t = g % p.ntiles;
+        q_pending |= 1u << stage;
+        mbar_arrive_expect_tx(&bQ[stage], IMG);
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh)
+            tma_load_3d(sQ + stage * IMG + kh * kRegion, &tmQ, &bQ[stage], kh * 64, t * kTile, bh);
+    };
+    // (leader) MMA1 S_p = Q C_par^T of tile g (its Q in stage `stage`), then the
+    // load of the next tile's Q into the other stage (free: every contraction
+    // that read it is complete); false when the wait for Q gave up
+    auto issue_mma1 = [&](int g, int stage) -> bool {
+        if (!wait_bar(&bQ[stage], (qph >> stage) & 1u, sAbort)) return false;
+        qph ^= 1u << stage;
+        q_pending &= ~(1u << stage);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks)
+            mma_ss(tmem, desc_k(sQ + stage * IMG, ks), desc_k(sCP, ks), idesc1, ks > 0);
+        mma_commit(bS);
+        if (g + 1 < g1) issue_q(g + 1, stage ^ 1);
+        return true;
+    };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        const uint32_t idesc1 = idesc_bf16_f32(128, p.M0p, false);
-        const uint32_t idesc3 = idesc_bf16_f32(128, D, true);
-        uint32_t wpph = 0, gph = 0, gtph = 0, wcph = 0, eph = 0;
-        auto issue_q = [&](int g, int stage) {
-            const int bh = g / p.ntiles, t = g % p.ntiles;
-            q_pending |= 1u << stage;
-            mbar_arrive_expect_tx(&bQ[stage], IMG);
-#pragma unroll
-            for (int kh = 0; kh < KH; ++kh)
-                tma_load_3d(sQ + stage * IMG + kh * kRegion, &tmQ, &bQ[stage], kh * 64, t * kTile, bh);
-        };
-        // MMA1 S_p = Q C_par^T of tile g (its Q in stage `stage`), then the load of
-        // the next tile's Q into the other stage (free: every contraction that
-        // read it has been issued before this one, and they run in order)
-        auto issue_mma1 = [&](int g, int stage) -> bool {
-            bool ok = wait_bar(&bQ[stage], (qph >> stage) & 1u, sAbort);
-            if (ok) {
-                qph ^= 1u << stage;
-                q_pending &= ~(1u << stage);
-            }
-            if (__any_sync(0xffffffffu, !ok)) return false;
-            if (lane == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < KSTEPS; ++ks)
-                    mma_ss(tmem, desc_k(sQ + stage * IMG, ks), desc_k(sCP, ks), idesc1, ks > 0);
-                mma_commit(bS);
-                if (g + 1 < g1) issue_q(g + 1, stage ^ 1);
-            }
-            __syncwarp();
-            return true;
-        };
-        auto load_head = [&](int bh) -> bool {   // this head's parent codewords and parent means
-            if (lane == 0) {
+    const int ct = tid;
+    const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
+    uint32_t sph = 0, oph = 0, cph = 0;
+    int cur_bh = -1;
+    bool mma1_chained = false;   // (leader) this tile's MMA1 went out at the end of the previous tile
+    const float2 sl2v = make_float2(p.sl2, p.sl2);
+    if (leader && g0 < g1) issue_q(g0, 0);
+    for (int g = g0, it = 0; g < g1; ++g, ++it) {
+        const int stage = it & 1;
+        const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
+        const int rows = min(kTile, p.N - t * kTile);
+        const bool valid = r < rows;
+        bool ok = true;
+        if (bh != cur_bh) {   // this (b,h)'s parent tables, log-counts and child counts
+            wg_sync();        // (every thread is past the previous tile, whose contractions are done)
+            if (leader) {     // parent codewords and parent means (TMA)
+                head_pending = true;
                 mbar_arrive_expect_tx(bHead, 2u * KH * (uint32_t)p.M0p * 128u);
 #pragma unroll
                 for (int kh = 0; kh < KH; ++kh) {
-                    tma_load_3d(sCP + kh * kRegion, &tmCB, bHead, kh * 64, 0, bh % p.H);
+                    tma_load_3d(sCP + kh * kRegion, &tmCB, bHead, kh * 64, 0, h);
                     tma_load_3d(sMP + kh * kRegion, &tmMN, bHead, kh * 64, 0, bh);
                 }
             }
-            head_pending = true;
-            bool ok = wait_bar(bHead, hph, sAbort);
-            if (ok) {
-                hph ^= 1;
-                head_pending = false;
+            __syncwarp();
+            if (ct < 128) {
+                const int n = ct < p.M0 ? __ldg(p.counts + (size_t)bh * p.Mtot + ct) : 0;
+                sLb[ct] = n > 0 ? __log2f((float)n) : -INFINITY;
+                sInvN[ct] = n > 0 ? 1.f / (float)n : 0.f;
             }
-            return !__any_sync(0xffffffffu, !ok);
-        };
-        if (lane == 0 && g0 < g1) issue_q(g0, 0);
-        __syncwarp();
-        bool mma1_done = false;   // the current tile's MMA1 was issued at the end of the previous one
-        for (int g = g0, it = 0; g < g1; ++g, ++it) {
-            const int stage = it & 1;
-            const int bh = g / p.ntiles;
-            bool ok = true;
-            if (!mma1_done) {
-                if (it > 0) {   // the previous tile's contractions are done (its O was read)
-                    ok = wait_bar(bEpi, eph, sAbort);
-                    eph ^= 1;
-                    if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
+            if (PC > 0)
+                for (int i = ct; i < p.M0 * C; i += 256) sCnt[i] = (float)__ldg(p.counts + (size_t)bh * p.Mtot + p.M0 + i);
+            wg_sync();
+            cur_bh = bh;
+        }
+        if (leader && !mma1_chained) {   // MMA1 S_p = Q C_par^T
+            if (head_pending) {
+                if (it == 0 && p.fail_first_wait) {   // (test hook) a wait whose limit is zero, and ran out
+                    ok = false;
+                    *sAbort = 1;
+                } else {
+                    ok = wait_bar(bHead, hph, sAbort);
                 }
-                if (!load_head(bh) || !issue_mma1(g, stage)) { failed = true; break; }
-            } else if (it > 0) {
-                ok = wait_bar(bEpi, eph, sAbort);   // (keeps the phase count; long complete)
-                eph ^= 1;
-                if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
+                if (ok) {
+                    hph ^= 1;
+                    head_pending = false;
+                }
             }
-            // the next tile's MMA1 can follow this tile's last contraction when it
-            // uses the same parent tables
-            const bool chain_next = g + 1 < g1 && (g + 1) / p.ntiles == bh;
-            if (it == 0 && p.fail_first_wait) {   // a wait whose limit is zero, and ran out
-                ok = false;
-                *sAbort = 1;
-            } else {
-                ok = wait_bar(bWp, wpph, sAbort);
+            ok = ok && issue_mma1(g, stage);
+        }
+        __syncwarp();   // (warp 0 converged again after its leader's part)
+        mma1_chained = false;
+        ok = wait_bar(bS, sph, sAbort) && ok;
+        sph ^= 1;
+        tc_fence_after();
+
+        // ---- parent pass over this thread's 16-column blocks 2i + hf:
+        // x_p = sl2 S_p + log2 n_p, the row's shift m, e'_p = 2^(x_p - m),
+        // Zbar (exact) and the denominator of the rounded weights. Two
+        // passes over S_p (the shift, then the weights), one block at a time.
+        float m, den;
+        {
+            const int nbp = (p.M0p / 16 + 1 - hf) / 2;   // this thread's parent blocks
+            float mp0 = -INFINITY, mp1 = -INFINITY;
+            for (int i = 0; i < nbp; ++i) {
+                const int b = 2 * i + hf;
+                float x[16];
+                tmem_ld16f(trow + 16 * b, x);
+                tmem_wait_ld();
+                tmem_touch16f(x);
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    const float4 lb = *reinterpret_cast<const float4*>(sLb + 16 * b + k);
+                    const float2 a2 = ffma2(make_float2(x[k], x[k + 1]), sl2v, make_float2(lb.x, lb.y));
+                    const float2 b2 = ffma2(make_float2(x[k + 2], x[k + 3]), sl2v, make_float2(lb.z, lb.w));
+                    mp0 = fmax3(mp0, a2.x, a2.y);
+                    mp1 = fmax3(mp1, b2.x, b2.y);
+                }
             }
-            wpph ^= 1;
-            if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
-            if (lane == 0) {   // MMA3p O = W_p x mean_par
+            sX[hf * 128 + r] = fmaxf(mp0, mp1);
+            pair_sync(q);
+            m = fmaxf(sX[r], sX[128 + r]);
+            const float2 negm = make_float2(-m, -m);
+            float2 z0 = make_float2(0.f, 0.f), z1 = make_float2(0.f, 0.f);
+            float2 zb0 = make_float2(0.f, 0.f), zb1 = make_float2(0.f, 0.f);
+            for (int i = 0; i < nbp; ++i) {
+                const int b = 2 * i + hf;
+                float x[16];
+                tmem_ld16f(trow + 16 * b, x);
+                tmem_wait_ld();
+                tmem_touch16f(x);
+                uint32_t w[8];
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    const float4 lb = *reinterpret_cast<const float4*>(sLb + 16 * b + k);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int o = k + 2 * e;
+                        const float2 xx = ffma2(make_float2(x[o], x[o + 1]), sl2v,
+                                                e ? make_float2(lb.z, lb.w) : make_float2(lb.x, lb.y));
+                        const float2 tt = fadd2(xx, negm);
+                        const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));
+                        x[o] = ev.x;
+                        x[o + 1] = ev.y;
+                        const uint32_t wb = pack_bf16x2(ev.x, ev.y);
+                        const float2 er = make_float2(bf16_lo(wb), bf16_hi(wb));
+                        if (e) { z1 = fadd2(z1, ev); zb1 = fadd2(zb1, er); }
+                        else { z0 = fadd2(z0, ev); zb0 = fadd2(zb0, er); }
+                        w[o >> 1] = wb;
+                    }
+                }
+                tmem_st8(trow + p.colWp + 8 * b, w);
+                if (PC > 0) tmem_st16f(trow + 16 * b, x);
+            }
+            sZ[hf * 128 + r] = (z0.x + z0.y) + (z1.x + z1.y);
+            den = (zb0.x + zb0.y) + (zb1.x + zb1.y);
+            pair_sync(q);
+            const float z = sZ[r] + sZ[128 + r];
+            sRz[r] = valid ? 1.f / z : 0.f;   // (both threads of the row write the same value)
+        }
+        tmem_wait_st();
+        tc_fence_before();   // (the W_p writes precede MMA3p, issued after a barrier)
+
+        if (PC > 0) {
+            // ---- importance w_p = sum over the tile's rows of e'_p / Zbar
+            // (each warp: its 32 rows, its four 16-column blocks)
+            __syncwarp();   // this warp's rows' 1/Zbar
+            {
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = 0.f;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int rlo = 32 * q + 16 * hh + (lane >> 2);
+                    const float2 rz = make_float2(sRz[rlo], sRz[rlo + 8]);
+                    float e[32];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int b = 2 * i + hf;
+                        if (16 * b < p.M0p) {
+                            tmem_ld_16x256b_x2(tmem + ((uint32_t)(32 * q + 16 * hh) << 16) + 16 * b, e + 8 * i);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) e[8 * i + k] = 0.f;
+                        }
+                    }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) touch8f(e + 8 * i);
+                    // register 4g + j of block 2i + hf: column 16(2i + hf) + 8g + 2(lane % 4) +
+                    // (j % 2) of row rlo (j < 2) or rlo + 8 (j >= 2); v index 4i + 2g + (j % 2)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int gg = 0; gg < 2; ++gg) {
+                            const float* ee = e + 8 * i + 4 * gg;
+                            float2 acc = make_float2(v[4 * i + 2 * gg], v[4 * i + 2 * gg + 1]);
+                            acc = ffma2(make_float2(ee[0], ee[1]), make_float2(rz.x, rz.x), acc);
+                            acc = ffma2(make_float2(ee[2], ee[3]), make_float2(rz.y, rz.y), acc);
+                            v[4 * i + 2 * gg] = acc.x;
+                            v[4 * i + 2 * gg + 1] = acc.y;
+                        }
+                }
+                // sum over the 8 lanes that hold the same columns (lane bits 2..4)
+                butterfly_level<8>(v, lane & 16, 16);
+                butterfly_level<4>(v, lane & 8, 8);
+                butterfly_level<2>(v, lane & 4, 4);
+                // v[e] = column 16(2i + hf) + 8g + 2(lane % 4) + e over the warp's rows,
+                // with i = (lane >> 3) & 3... : lane bits 4, 3 give i, bit 2 gives g
+                const int ii = 2 * ((lane >> 4) & 1) + ((lane >> 3) & 1), gg = (lane >> 2) & 1;
+                const int c0 = 16 * (2 * ii + hf) + 8 * gg + 2 * (lane & 3);
+                *reinterpret_cast<float2*>(sPart + q * 128 + c0) = make_float2(v[0], v[1]);
+            }
+            tc_fence_before();   // the reads of e' precede MMA2 (issued after later barriers)
+            if (wg_sync_or(!ok)) { failed = true; break; }
+            if (leader) {   // MMA3p O = W_p x mean_par (W_p is complete)
                 tc_fence_after();
                 for (int ks = 0; ks < p.M0p / 16; ++ks)
                     mma_ts(tmem + p.colO, tmem + p.colWp + 8 * ks, desc_mn(sMP, ks), idesc3, ks > 0);
-                if (nchunks == 0) mma_commit(bO);
             }
             __syncwarp();
-            for (int k = 0; k < nchunks; ++k) {
-                const int N2 = (min(128, PC - 128 * k) + 15) & ~15;
-                if (tma_gather) {                   // the chunk's children are in shared memory
-                    ok = wait_bar(bGatT, gtph, sAbort);
-                    gtph ^= 1;
-                } else {
-                    ok = wait_bar(bGat, gph, sAbort);
-                    gph ^= 1;
-                }
-                if (__any_sync(0xffffffffu, !ok)) break;
-                if (lane == 0) {   // MMA2 S_c = Q C_child^T
-                    tc_fence_after();
-                    const uint32_t idesc2 = idesc_bf16_f32(128, N2, false);
+
+            // ---- top-P: the parents ordered by (importance, then the lower
+            // index), the first P selected in rank order (select_top_p4)
+            if (hf == 0)
+                select_top_p4(sPart, reinterpret_cast<unsigned long long*>(sX), sSel,
+                              p.selected + ((size_t)bh * p.ntiles + t) * p.P, p.M0, p.P, q, lane);
+            if (store_thread) bulk_wait_read_all();   // the previous O store has read the staging
+            wg_sync();   // the selection is in sSel
+            gat_pending = tma_gather;   // (leader: the gather below is in flight until bGatT completes)
+            {
+                if (tma_gather) {   // each selected parent's children: one TMA load per image
+                    // (slot s from thread 32 (s % 8) + s / 8: the loads leave from all
+                    // eight warps, not one warp's lanes in turn)
+                    const int gslot = (ct & 31) * 8 + (ct >> 5);
+                    if (gslot < p.P) {
+                        const int par = min(max(sSel[gslot], 0), p.M0 - 1);
+                        mbar_arrive_expect_tx(bGatT, 2u * KH * (uint32_t)C * 128u);
 #pragma unroll
-                    for (int ks = 0; ks < KSTEPS; ++ks)
-                        mma_ss(tmem, desc_k(sQ + stage * IMG, ks), desc_k(sCC, ks), idesc2, ks > 0);
-                    mma_commit(bS);
+                        for (int kh = 0; kh < KH; ++kh) {
+                            tma_load_3d(sCC + kh * kRegion + gslot * C * 128, &tmCBc, bGatT, kh * 64, p.M0 + par * C, h);
+                            tma_load_3d(sMC + kh * kRegion + gslot * C * 128, &tmMNc, bGatT, kh * 64, p.M0 + par * C, bh);
+                        }
+                    }
+                    if (ct < PC) {   // slot tables: the child's count and its log2
+                        const float nc = sCnt[min(max(sSel[ct / C], 0), p.M0 - 1) * C + ct % C];
+                        sNc[ct] = nc;
+                        sLc[ct] = nc > 0.f ? __log2f(nc) : -INFINITY;
+                    }
                 }
-                ok = wait_bar(bWc, wcph, sAbort);
-                wcph ^= 1;
-                if (__any_sync(0xffffffffu, !ok)) break;
-                if (lane == 0) {   // MMA3c O += W_c x mean_child (the last chunk's W_c is over W_p)
+                if (tma_gather && ct == 255) {   // the chunk's padding slots: zero rows, empty entries
+                    const int N2 = (PC + 15) & ~15;
+                    for (int slot = PC; slot < N2; ++slot) {
+                        sNc[slot] = 0.f;
+                        sLc[slot] = -INFINITY;
+#pragma unroll
+                        for (int j = 0; j < D / 8; ++j) {
+                            *reinterpret_cast<uint4*>(sCC + swz(slot, j)) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(sMC + swz(slot, j)) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(bGatT);
+                }
+            }
+
+            // ---- children, chunk by chunk
+            for (int k = 0; k < nchunks; ++k) {
+                const int cs = 128 * k;
+                const int ns = min(128, PC - cs);
+                const int N2 = (ns + 15) & ~15;
+                if (!tma_gather) {
+                if (k > 0) {
+                    ok = wait_bar(bC, cph, sAbort) && ok;      // the previous chunk's MMA3c is done
+                    cph ^= 1;
+                }
+                wg_sync();   // the selection is complete; the previous chunk's tables are no longer read
+                // slot tables and the gather of the chunk's child codewords and value means
+                if (ct < N2) {
+                    float nc = 0.f;
+                    if (ct < ns) {
+                        const int sg = cs + ct;
+                        nc = sCnt[min(max(sSel[sg / C], 0), p.M0 - 1) * C + (sg % C)];
+                    }
+                    sNc[ct] = nc;
+                    sLc[ct] = nc > 0.f ? __log2f(nc) : -INFINITY;
+                }
+                for (int idx = ct; idx < N2 * (D / 8); idx += 256) {
+                    const int slot = idx / (D / 8), j = idx % (D / 8);
+                    const uint32_t off = swz(slot, j);
+                    if (slot < ns) {
+                        const int sg = cs + slot;
+                        const int child = p.M0 + min(max(sSel[sg / C], 0), p.M0 - 1) * C + (sg % C);
+                        cp_async_16(sCC + off, p.codebook + ((size_t)h * p.Mtot + child) * D + j * 8);
+                        cp_async_16(sMC + off, p.means + ((size_t)bh * p.Mtot + child) * D + j * 8);
+                    } else {
+                        *reinterpret_cast<uint4*>(sCC + off) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(sMC + off) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                wg_sync();   // the chunk's children are in shared memory
+                }
+                if (leader) {   // MMA2 S_c = Q C_child^T
+                    if (tma_gather) {
+                        ok = wait_bar(bGatT, gtph, sAbort) && ok;
+                        if (ok) {
+                            gtph ^= 1;
+                            gat_pending = false;
+                        }
+                    }
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t idesc2 = idesc_bf16_f32(128, N2, false);
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks)
+                            mma_ss(tmem, desc_k(sQ + stage * IMG, ks), desc_k(sCC, ks), idesc2, ks > 0);
+                        mma_commit(bS);
+                    } else {
+                        *sAbort = 1;   // (the others' wait for S_c gives up too)
+                    }
+                }
+                __syncwarp();
+                ok = wait_bar(bS, sph, sAbort) && ok;
+                sph ^= 1;
+                tc_fence_after();
+                wg_sync();           // the slot tables and the selection are complete
+                // child weights (A_c - A_p) n_c = 2^t - A_p n_c with t = sl2 S_c +
+                // log2 n_c - m, over this thread's 16-slot blocks 2i + hf, rounded to
+                // bf16 once; the denominator from the same rounded values. They are
+                // held until both threads of the row have read their S_c, then
+                // written as W_c over the S_c columns. When the row's largest t is
+                // above 64 the shift moves up by whole octaves: O, W_p and the
+                // denominator are scaled by 2^-k (exact) and the weights taken again
+                // (paper §4.3: the running accumulators follow the maximum).
+                const int nb = (N2 / 16 + 1 - hf) / 2;
+                float2 dc0, dc1;
+                uint32_t wall[4][8];
+#pragma unroll 1
+                for (int attempt = 0;; ++attempt) {
+                    const float2 negm = make_float2(-m, -m);
+                    float tmax = -INFINITY;
+                    dc0 = make_float2(0.f, 0.f);
+                    dc1 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (i >= nb) break;
+                        const int b = 2 * i + hf;
+                        constexpr int PB = C >= 16 ? 1 : 16 / C;   // parents behind a 16-slot block
+                        float sc[16];
+                        float nap[PB];
+                        {
+                            int pid[PB];
+                            uint32_t wr[PB];
+                            tmem_ld16f(trow + 16 * b, sc);
+#pragma unroll
+                            for (int j = 0; j < PB; ++j) {
+                                pid[j] = min(max(sSel[min((cs + 16 * b) / C + j, p.P - 1)], 0), p.M0 - 1);
+                                tmem_ld1(trow + p.colWp + (pid[j] >> 1), wr[j]);
+                            }
+                            tmem_wait_ld();
+                            tmem_touch16f(sc);
+#pragma unroll
+                            for (int j = 0; j < PB; ++j) {
+                                tmem_touch1(wr[j]);
+                                nap[j] = -((pid[j] & 1) ? bf16_hi(wr[j]) : bf16_lo(wr[j])) * sInvN[pid[j]];
+                            }
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < 16; kk += 4) {
+                            const float4 lc = *reinterpret_cast<const float4*>(sLc + 16 * b + kk);
+                            const float4 nc = *reinterpret_cast<const float4*>(sNc + 16 * b + kk);
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int s = kk + 2 * e;
+                                const float2 tt = ffma2(make_float2(sc[s], sc[s + 1]), sl2v,
+                                                        fadd2(e ? make_float2(lc.z, lc.w) : make_float2(lc.x, lc.y), negm));
+                                tmax = fmax3(tmax, tt.x, tt.y);
+                                const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));
+                                const float2 wc = ffma2(make_float2(nap[s / C < PB ? s / C : 0], nap[(s + 1) / C < PB ? (s + 1) / C : 0]),
+                                                        e ? make_float2(nc.z, nc.w) : make_float2(nc.x, nc.y), ev);
+                                const uint32_t wb = pack_bf16x2(wc.x, wc.y);
+                                const float2 wr2 = make_float2(bf16_lo(wb), bf16_hi(wb));
+                                if (e) dc1 = fadd2(dc1, wr2);
+                                else dc0 = fadd2(dc0, wr2);
+                                wall[i][s >> 1] = wb;
+                            }
+                        }
+                    }
+                    sT[hf * 128 + r] = tmax;
+                    pair_sync(q);   // both threads' S_c and W_p reads precede any write to them
+                    tmax = fmaxf(sT[r], sT[128 + r]);
+                    const bool up = attempt == 0 && tmax > kRescale;
+                    if (!__any_sync(0xffffffffu, up)) break;
+                    // (rare) The TMEM accesses are warp-collective: rows that keep
+                    // their shift take factor 1.
+                    const int kup = up ? (int)ceilf(fminf(tmax, 1.0e6f)) : 0;
+                    const float f = exp2_neg_int(kup);
+                    m += (float)kup;
+                    den *= f;
+                    for (int c = 0; c < OD / 16; ++c) {   // this thread's half of O
+                        float o[16];
+                        tmem_ld16f(trow + p.colO + hf * OD + 16 * c, o);
+                        tmem_wait_ld();
+                        tmem_touch16f(o);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] *= f;
+                        tmem_st16f(trow + p.colO + hf * OD + 16 * c, o);
+                    }
+                    for (int i = 0; i < 4; ++i) {         // this thread's blocks of W_p
+                        const int b = 2 * i + hf;
+                        if (16 * b >= p.M0p) break;
+                        uint32_t u[8];
+                        tmem_ld8(trow + p.colWp + 8 * b, u);
+                        tmem_wait_ld();
+                        touch8u(u);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) u[j] = pack_bf16x2(bf16_lo(u[j]) * f, bf16_hi(u[j]) * f);
+                        tmem_st8(trow + p.colWp + 8 * b, u);
+                    }
+                    tmem_wait_st();
+                    pair_sync(q);   // the partner's blocks of W_p are scaled too
+                }
+                // W_c goes over the chunk's S_c columns, except for the tile's last
+                // chunk: that one goes over W_p (no lookup needs it any more), so
+                // that the next tile's MMA1 may write the S columns while the last
+                // MMA3c still reads W_c
+                const uint32_t colWc = k + 1 == nchunks ? p.colWp : 0u;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (i >= nb) break;
+                    tmem_st8(trow + colWc + 8 * (2 * i + hf), wall[i]);
+                }
+                den += (dc0.x + dc0.y) + (dc1.x + dc1.y);
+                tmem_wait_st();
+                tc_fence_before();
+                if (wg_sync_or(!ok)) { failed = true; break; }
+                if (leader) {   // MMA3c O += W_c x mean_child (the last chunk's W_c is over W_p)
                     tc_fence_after();
-                    const uint32_t colWc = k + 1 == nchunks ? p.colWp : 0u;
                     for (int ks = 0; ks < N2 / 16; ++ks)
                         mma_ts(tmem + p.colO, tmem + colWc + 8 * ks, desc_mn(sMC, ks), idesc3, 1);
                     mma_commit(k + 1 < nchunks ? bC : bO);
                 }
                 __syncwarp();
             }
-            if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
-            // (the compute threads have read every S column of this tile and the
-            // contractions above read no S column: the next MMA1 may write them)
-            mma1_done = false;
-            if (chain_next) {
-                if (!issue_mma1(g + 1, stage ^ 1)) { failed = true; break; }
-                mma1_done = true;
+            if (failed) break;
+        } else {
+            if (wg_sync_or(!ok)) { failed = true; break; }
+            if (leader) {   // MMA3p O = W_p x mean_par, the tile's only value contraction
+                tc_fence_after();
+                for (int ks = 0; ks < p.M0p / 16; ++ks)
+                    mma_ts(tmem + p.colO, tmem + p.colWp + 8 * ks, desc_mn(sMP, ks), idesc3, ks > 0);
+                mma_commit(bO);
             }
+            __syncwarp();
         }
-    } else {
-        // ------------------------------------------------------ compute rows
-        const int ct = tid - 32;                      // 0 .. 255
-        const int q = warp & 3;                       // TMEM lane quarter of this warp
-        const int hf = (warp - 1) >> 2;               // which half of the row's columns
-        const int r = 32 * q + lane;                  // query row (and parent / slot index)
-        const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
-        const bool store_thread = tid == 32;
-        uint32_t sph = 0, oph = 0, cph = 0;
-        int cur_bh = -1;
-        const float2 sl2v = make_float2(p.sl2, p.sl2);
-        for (int g = g0; g < g1; ++g) {
-            const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
-            const int rows = min(kTile, p.N - t * kTile);
-            const bool valid = r < rows;
-            if (bh != cur_bh) {   // this (b,h)'s parent log-counts and child counts
-                wg_sync();        // (every thread is past its last use of the previous ones)
-                if (ct < 128) {
-                    const int n = ct < p.M0 ? __ldg(p.counts + (size_t)bh * p.Mtot + ct) : 0;
-                    sLb[ct] = n > 0 ? __log2f((float)n) : -INFINITY;
-                    sInvN[ct] = n > 0 ? 1.f / (float)n : 0.f;
-                }
-                if (PC > 0)
-                    for (int i = ct; i < p.M0 * C; i += 256) sCnt[i] = (float)__ldg(p.counts + (size_t)bh * p.Mtot + p.M0 + i);
-                wg_sync();
-                cur_bh = bh;
-            }
-            bool ok = wait_bar(bS, sph, sAbort);
-            sph ^= 1;
-            tc_fence_after();
+        // the next tile's MMA1 follows this tile's last contraction when it uses
+        // the same parent tables (every S column of this tile has been read, and
+        // no contraction above reads one)
+        if (leader && g + 1 < g1 && (g + 1) / p.ntiles == bh) {
+            if (issue_mma1(g + 1, stage ^ 1)) mma1_chained = true;
+            else ok = false;   // (seen by everyone at the barrier below)
+        }
+        __syncwarp();
 
-            // ---- parent pass over this thread's 16-column blocks 2i + hf:
-            // x_p = sl2 S_p + log2 n_p, the row's shift m, e'_p = 2^(x_p - m),
-            // Zbar (exact) and the denominator of the rounded weights. Two
-            // passes over S_p (the shift, then the weights), one block at a time.
-            float m, den;
-            {
-                const int nbp = (p.M0p / 16 + 1 - hf) / 2;   // this thread's parent blocks
-                float mp0 = -INFINITY, mp1 = -INFINITY;
-                for (int i = 0; i < nbp; ++i) {
-                    const int b = 2 * i + hf;
-                    float x[16];
-                    tmem_ld16f(trow + 16 * b, x);
-                    tmem_wait_ld();
-                    tmem_touch16f(x);
+        // ---- epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
+        // (this thread: output dimensions hf * OD .. hf * OD + OD - 1)
+        sZ[hf * 128 + r] = den;
+        ok = wait_bar(bO, oph, sAbort) && ok;
+        oph ^= 1;
+        tc_fence_after();
+        uint32_t packed[OD / 2];
+        {
+            float o[OD];
 #pragma unroll
-                    for (int k = 0; k < 16; k += 4) {
-                        const float4 lb = *reinterpret_cast<const float4*>(sLb + 16 * b + k);
-                        const float2 a2 = ffma2(make_float2(x[k], x[k + 1]), sl2v, make_float2(lb.x, lb.y));
-                        const float2 b2 = ffma2(make_float2(x[k + 2], x[k + 3]), sl2v, make_float2(lb.z, lb.w));
-                        mp0 = fmax3(mp0, a2.x, a2.y);
-                        mp1 = fmax3(mp1, b2.x, b2.y);
-                    }
-                }
-                sX[hf * 128 + r] = fmaxf(mp0, mp1);
-                pair_sync(q);
-                m = fmaxf(sX[r], sX[128 + r]);
-                const float2 negm = make_float2(-m, -m);
-                float2 z0 = make_float2(0.f, 0.f), z1 = make_float2(0.f, 0.f);
-                float2 zb0 = make_float2(0.f, 0.f), zb1 = make_float2(0.f, 0.f);
-                for (int i = 0; i < nbp; ++i) {
-                    const int b = 2 * i + hf;
-                    float x[16];
-                    tmem_ld16f(trow + 16 * b, x);
-                    tmem_wait_ld();
-                    tmem_touch16f(x);
-                    uint32_t w[8];
+            for (int c = 0; c < OD / 16; ++c) tmem_ld16f(trow + p.colO + hf * OD + 16 * c, o + 16 * c);
+            tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 16; k += 4) {
-                        const float4 lb = *reinterpret_cast<const float4*>(sLb + 16 * b + k);
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int o = k + 2 * e;
-                            const float2 xx = ffma2(make_float2(x[o], x[o + 1]), sl2v,
-                                                    e ? make_float2(lb.z, lb.w) : make_float2(lb.x, lb.y));
-                            const float2 tt = fadd2(xx, negm);
-                            const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));
-                            x[o] = ev.x;
-                            x[o + 1] = ev.y;
-                            const uint32_t wb = pack_bf16x2(ev.x, ev.y);
-                            const float2 er = make_float2(bf16_lo(wb), bf16_hi(wb));
-                            if (e) { z1 = fadd2(z1, ev); zb1 = fadd2(zb1, er); }
-                            else { z0 = fadd2(z0, ev); zb0 = fadd2(zb0, er); }
-                            w[o >> 1] = wb;
-                        }
-                    }
-                    tmem_st8(trow + p.colWp + 8 * b, w);
-                    if (PC > 0) tmem_st16f(trow + 16 * b, x);
-                }
-                sZ[hf * 128 + r] = (z0.x + z0.y) + (z1.x + z1.y);
-                den = (zb0.x + zb0.y) + (zb1.x + zb1.y);
-                pair_sync(q);
-                const float z = sZ[r] + sZ[128 + r];
-                sRz[r] = valid ? 1.f / z : 0.f;   // (both threads of the row write the same value)
-            }
-            tmem_wait_st();
+            for (int c = 0; c < OD / 16; ++c) tmem_touch16f(o + 16 * c);
             tc_fence_before();
-            mbar_arrive(bWp);
-
-            if (PC > 0) {
-                // ---- importance w_p = sum over the tile's rows of e'_p / Zbar
-                // (each warp: its 32 rows, its four 16-column blocks)
-                __syncwarp();   // this warp's rows' 1/Zbar
-                {
-                    float v[16];
+            pair_sync(q);
+            const float inv = 1.f / (sZ[r] + sZ[128 + r]);
+            const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int rlo = 32 * q + 16 * hh + (lane >> 2);
-                        const float2 rz = make_float2(sRz[rlo], sRz[rlo + 8]);
-                        float e[32];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int b = 2 * i + hf;
-                            if (16 * b < p.M0p) {
-                                tmem_ld_16x256b_x2(tmem + ((uint32_t)(32 * q + 16 * hh) << 16) + 16 * b, e + 8 * i);
-                            } else {
-#pragma unroll
-                                for (int k = 0; k < 8; ++k) e[8 * i + k] = 0.f;
-                            }
-                        }
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) touch8f(e + 8 * i);
-                        // register 4g + j of block 2i + hf: column 16(2i + hf) + 8g + 2(lane % 4) +
-                        // (j % 2) of row rlo (j < 2) or rlo + 8 (j >= 2); v index 4i + 2g + (j % 2)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-#pragma unroll
-                            for (int gg = 0; gg < 2; ++gg) {
-                                const float* ee = e + 8 * i + 4 * gg;
-                                float2 acc = make_float2(v[4 * i + 2 * gg], v[4 * i + 2 * gg + 1]);
-                                acc = ffma2(make_float2(ee[0], ee[1]), make_float2(rz.x, rz.x), acc);
-                                acc = ffma2(make_float2(ee[2], ee[3]), make_float2(rz.y, rz.y), acc);
-                                v[4 * i + 2 * gg] = acc.x;
-                                v[4 * i + 2 * gg + 1] = acc.y;
-                            }
-                    }
-                    // sum over the 8 lanes that hold the same columns (lane bits 2..4)
-                    butterfly_level<8>(v, lane & 16, 16);
-                    butterfly_level<4>(v, lane & 8, 8);
-                    butterfly_level<2>(v, lane & 4, 4);
-                    // v[e] = column 16(2i + hf) + 8g + 2(lane % 4) + e over the warp's rows,
-                    // with i = (lane >> 3) & 3... : lane bits 4, 3 give i, bit 2 gives g
-                    const int ii = 2 * ((lane >> 4) & 1) + ((lane >> 3) & 1), gg = (lane >> 2) & 1;
-                    const int c0 = 16 * (2 * ii + hf) + 8 * gg + 2 * (lane & 3);
-                    *reinterpret_cast<float2*>(sPart + q * 128 + c0) = make_float2(v[0], v[1]);
-                }
-                tc_fence_before();   // the reads of e' precede MMA2 (issued after later hand-overs)
-                if (wg_sync_or(!ok)) { failed = true; break; }
-
-                // ---- top-P: the parents ordered by (importance, then the lower
-                // index), the first P selected in rank order (select_top_p4)
-                if (hf == 0)
-                    select_top_p4(sPart, reinterpret_cast<unsigned long long*>(sX), sSel,
-                                  p.selected + ((size_t)bh * p.ntiles + t) * p.P, p.M0, p.P, q, lane);
-                if (store_thread) bulk_wait_read_all();   // the previous O store has read the staging
-                wg_sync();   // the selection is in sSel
-                {
-                    if (tma_gather) {   // each selected parent's children: one TMA load per image
-                        // (slot s from thread 32 (s % 8) + s / 8: the loads leave from all
-                        // eight warps, not one warp's lanes in turn)
-                        const int gslot = (ct & 31) * 8 + (ct >> 5);
-                        if (gslot < p.P) {
-                            const int par = min(max(sSel[gslot], 0), p.M0 - 1);
-                            mbar_arrive_expect_tx(bGatT, 2u * KH * (uint32_t)C * 128u);
-#pragma unroll
-                            for (int kh = 0; kh < KH; ++kh) {
-                                tma_load_3d(sCC + kh * kRegion + gslot * C * 128, &tmCBc, bGatT, kh * 64, p.M0 + par * C, h);
-                                tma_load_3d(sMC + kh * kRegion + gslot * C * 128, &tmMNc, bGatT, kh * 64, p.M0 + par * C, bh);
-                            }
-                        }
-                        if (ct < PC) {   // slot tables: the child's count and its log2
-                            const float nc = sCnt[min(max(sSel[ct / C], 0), p.M0 - 1) * C + ct % C];
-                            sNc[ct] = nc;
-                            sLc[ct] = nc > 0.f ? __log2f(nc) : -INFINITY;
-                        }
-                    }
-                    if (tma_gather && ct == 255) {   // the chunk's padding slots: zero rows, empty entries
-                        const int N2 = (PC + 15) & ~15;
-                        for (int slot = PC; slot < N2; ++slot) {
-                            sNc[slot] = 0.f;
-                            sLc[slot] = -INFINITY;
-#pragma unroll
-                            for (int j = 0; j < D / 8; ++j) {
-                                *reinterpret_cast<uint4*>(sCC + swz(slot, j)) = make_uint4(0, 0, 0, 0);
-                                *reinterpret_cast<uint4*>(sMC + swz(slot, j)) = make_uint4(0, 0, 0, 0);
-                            }
-                        }
-                        fence_proxy_async_smem();
-                        mbar_arrive(bGatT);
-                    }
-                }
-
-                // ---- children, chunk by chunk
-                for (int k = 0; k < nchunks; ++k) {
-                    const int cs = 128 * k;
-                    const int ns = min(128, PC - cs);
-                    const int N2 = (ns + 15) & ~15;
-                    if (!tma_gather) {
-                    if (k > 0) {
-                        ok = wait_bar(bC, cph, sAbort) && ok;      // the previous chunk's MMA3c is done
-                        cph ^= 1;
-                    }
-                    wg_sync();   // the selection is complete; the previous chunk's tables are no longer read
-                    // slot tables and the gather of the chunk's child codewords and value means
-                    if (ct < N2) {
-                        float nc = 0.f;
-                        if (ct < ns) {
-                            const int sg = cs + ct;
-                            nc = sCnt[min(max(sSel[sg / C], 0), p.M0 - 1) * C + (sg % C)];
-                        }
-                        sNc[ct] = nc;
-                        sLc[ct] = nc > 0.f ? __log2f(nc) : -INFINITY;
-                    }
-                    for (int idx = ct; idx < N2 * (D / 8); idx += 256) {
-                        const int slot = idx / (D / 8), j = idx % (D / 8);
-                        const uint32_t off = swz(slot, j);
-                        if (slot < ns) {
-                            const int sg = cs + slot;
-                            const int child = p.M0 + min(max(sSel[sg / C], 0), p.M0 - 1) * C + (sg % C);
-                            cp_async_16(sCC + off, p.codebook + ((size_t)h * p.Mtot + child) * D + j * 8);
-                            cp_async_16(sMC + off, p.means + ((size_t)bh * p.Mtot + child) * D + j * 8);
-                        } else {
-                            *reinterpret_cast<uint4*>(sCC + off) = make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4*>(sMC + off) = make_uint4(0, 0, 0, 0);
-                        }
-                    }
-                    cp_async_wait_all();
-                    fence_proxy_async_smem();
-                    tc_fence_before();   // (chunk 0) the importance's reads of e' precede MMA2
-                    mbar_arrive(bGat);
-                    }
-                    ok = wait_bar(bS, sph, sAbort) && ok;
-                    sph ^= 1;
-                    tc_fence_after();
-                    wg_sync();           // the slot tables and the selection are complete
-                    // child weights (A_c - A_p) n_c = 2^t - A_p n_c with t = sl2 S_c +
-                    // log2 n_c - m, over this thread's 16-slot blocks 2i + hf, rounded to
-                    // bf16 once; the denominator from the same rounded values. They are
-                    // held until both threads of the row have read their S_c, then
-                    // written as W_c over the S_c columns. When the row's largest t is
-                    // above 64 the shift moves up by whole octaves: O, W_p and the
-                    // denominator are scaled by 2^-k (exact) and the weights taken again
-                    // (paper §4.3: the running accumulators follow the maximum).
-                    const int nb = (N2 / 16 + 1 - hf) / 2;
-                    float2 dc0, dc1;
-                    uint32_t wall[4][8];
-#pragma unroll 1
-                    for (int attempt = 0;; ++attempt) {
-                        const float2 negm = make_float2(-m, -m);
-                        float tmax = -INFINITY;
-                        dc0 = make_float2(0.f, 0.f);
-                        dc1 = make_float2(0.f, 0.f);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            if (i >= nb) break;
-                            const int b = 2 * i + hf;
-                            constexpr int PB = C >= 16 ? 1 : 16 / C;   // parents behind a 16-slot block
-                            float sc[16];
-                            float nap[PB];
-                            {
-                                int pid[PB];
-                                uint32_t wr[PB];
-                                tmem_ld16f(trow + 16 * b, sc);
-#pragma unroll
-                                for (int j = 0; j < PB; ++j) {
-                                    pid[j] = min(max(sSel[min((cs + 16 * b) / C + j, p.P - 1)], 0), p.M0 - 1);
-                                    tmem_ld1(trow + p.colWp + (pid[j] >> 1), wr[j]);
-                                }
-                                tmem_wait_ld();
-                                tmem_touch16f(sc);
-#pragma unroll
-                                for (int j = 0; j < PB; ++j) {
-                                    tmem_touch1(wr[j]);
-                                    nap[j] = -((pid[j] & 1) ? bf16_hi(wr[j]) : bf16_lo(wr[j])) * sInvN[pid[j]];
-                                }
-                            }
-#pragma unroll
-                            for (int kk = 0; kk < 16; kk += 4) {
-                                const float4 lc = *reinterpret_cast<const float4*>(sLc + 16 * b + kk);
-                                const float4 nc = *reinterpret_cast<const float4*>(sNc + 16 * b + kk);
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int s = kk + 2 * e;
-                                    const float2 tt = ffma2(make_float2(sc[s], sc[s + 1]), sl2v,
-                                                            fadd2(e ? make_float2(lc.z, lc.w) : make_float2(lc.x, lc.y), negm));
-                                    tmax = fmax3(tmax, tt.x, tt.y);
-                                    const float2 ev = make_float2(ex2(tt.x), ex2(tt.y));
-                                    const float2 wc = ffma2(make_float2(nap[s / C < PB ? s / C : 0], nap[(s + 1) / C < PB ? (s + 1) / C : 0]),
-                                                            e ? make_float2(nc.z, nc.w) : make_float2(nc.x, nc.y), ev);
-                                    const uint32_t wb = pack_bf16x2(wc.x, wc.y);
-                                    const float2 wr2 = make_float2(bf16_lo(wb), bf16_hi(wb));
-                                    if (e) dc1 = fadd2(dc1, wr2);
-                                    else dc0 = fadd2(dc0, wr2);
-                                    wall[i][s >> 1] = wb;
-                                }
-                            }
-                        }
-                        sT[hf * 128 + r] = tmax;
-                        pair_sync(q);   // both threads' S_c and W_p reads precede any write to them
-                        tmax = fmaxf(sT[r], sT[128 + r]);
-                        const bool up = attempt == 0 && tmax > kRescale;
-                        if (!__any_sync(0xffffffffu, up)) break;
-                        // (rare) The TMEM accesses are warp-collective: rows that keep
-                        // their shift take factor 1.
-                        const int kup = up ? (int)ceilf(fminf(tmax, 1.0e6f)) : 0;
-                        const float f = exp2_neg_int(kup);
-                        m += (float)kup;
-                        den *= f;
-                        for (int c = 0; c < OD / 16; ++c) {   // this thread's half of O
-                            float o[16];
-                            tmem_ld16f(trow + p.colO + hf * OD + 16 * c, o);
-                            tmem_wait_ld();
-                            tmem_touch16f(o);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) o[i] *= f;
-                            tmem_st16f(trow + p.colO + hf * OD + 16 * c, o);
-                        }
-                        for (int i = 0; i < 4; ++i) {         // this thread's blocks of W_p
-                            const int b = 2 * i + hf;
-                            if (16 * b >= p.M0p) break;
-                            uint32_t u[8];
-                            tmem_ld8(trow + p.colWp + 8 * b, u);
-                            tmem_wait_ld();
-                            touch8u(u);
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) u[j] = pack_bf16x2(bf16_lo(u[j]) * f, bf16_hi(u[j]) * f);
-                            tmem_st8(trow + p.colWp + 8 * b, u);
-                        }
-                        tmem_wait_st();
-                        pair_sync(q);   // the partner's blocks of W_p are scaled too
-                    }
-                    // W_c goes over the chunk's S_c columns, except for the tile's last
-                    // chunk: that one goes over W_p (no lookup needs it any more), so
-                    // that the next tile's MMA1 may write the S columns while the last
-                    // MMA3c still reads W_c
-                    const uint32_t colWc = k + 1 == nchunks ? p.colWp : 0u;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (i >= nb) break;
-                        tmem_st8(trow + colWc + 8 * (2 * i + hf), wall[i]);
-                    }
-                    den += (dc0.x + dc0.y) + (dc1.x + dc1.y);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(bWc);
-                }
-            }
-
-            // ---- epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
-            // (this thread: output dimensions hf * OD .. hf * OD + OD - 1)
-            sZ[hf * 128 + r] = den;
-            ok = wait_bar(bO, oph, sAbort) && ok;
-            oph ^= 1;
-            tc_fence_after();
-            uint32_t packed[OD / 2];
-            {
-                float o[OD];
-#pragma unroll
-                for (int c = 0; c < OD / 16; ++c) tmem_ld16f(trow + p.colO + hf * OD + 16 * c, o + 16 * c);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < OD / 16; ++c) tmem_touch16f(o + 16 * c);
-                tc_fence_before();
-                mbar_arrive(bEpi);
-                pair_sync(q);
-                const float inv = 1.f / (sZ[r] + sZ[128 + r]);
-                const float2 inv2 = make_float2(inv, inv);
-#pragma unroll
-                for (int i = 0; i < OD / 2; ++i) {
-                    const float2 v2 = fmul2(make_float2(o[2 * i], o[2 * i + 1]), inv2);
-                    packed[i] = pack_bf16x2(v2.x, v2.y);
-                }
-            }
-            if (PC == 0 && store_thread) bulk_wait_read_all();
-            if (wg_sync_or(!ok)) { failed = true; break; }   // the staging buffer is free
-#pragma unroll
-            for (int j = 0; j < OD / 8; ++j)
-                *reinterpret_cast<uint4*>(sMC + swz(r, hf * (OD / 8) + j)) =
-                    make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-            fence_proxy_async_smem();
-            wg_sync();
-            if (store_thread) {
-#pragma unroll
-                for (int kh = 0; kh < KH; ++kh) tma_store_3d(&tmO, sMC + kh * kRegion, kh * 64, t * kTile, bh);
-                bulk_commit();
+            for (int i = 0; i < OD / 2; ++i) {
+                const float2 v2 = fmul2(make_float2(o[2 * i], o[2 * i + 1]), inv2);
+                packed[i] = pack_bf16x2(v2.x, v2.y);
             }
         }
-        cp_async_wait_all();
-        if (store_thread) bulk_wait_all();
+        if (PC == 0 && store_thread) bulk_wait_read_all();
+        if (wg_sync_or(!ok)) { failed = true; break; }   // the staging buffer is free
+#pragma unroll
+        for (int j = 0; j < OD / 8; ++j)
+            *reinterpret_cast<uint4*>(sMC + swz(r, hf * (OD / 8) + j)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        fence_proxy_async_smem();
+        wg_sync();
+        if (store_thread) {
+#pragma unroll
+            for (int kh = 0; kh < KH; ++kh) tma_store_3d(&tmO, sMC + kh * kRegion, kh * 64, t * kTile, bh);
+            bulk_commit();
+        }
     }
+    cp_async_wait_all();
+    if (store_thread) bulk_wait_all();
 
-    if (failed && (tid == 0 || tid == 32)) {
+    if (failed && tid == 0) {
         atomicExch(&p.status->error, (int)AVQ_ETIMEOUT);
         atomicExch(&p.status->where, (int)blockIdx.x);
     }
-    if (failed && tid == 0) {
+    if (failed && leader) {
         // contractions and loads still in flight finish before the TMEM and the
         // shared memory go back (each wait bounded)
         mma_commit(bFin);
@@ -881,6 +830,7 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         for (int st = 0; st < 2; ++st)
             if (q_pending & (1u << st)) mbar_wait(&bQ[st], (qph >> st) & 1u);
         if (head_pending) mbar_wait(bHead, hph);
+        if (gat_pending) mbar_wait(bGatT, gtph);
     }
     tc_fence_before();
     __syncthreads();
@@ -891,9 +841,9 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 }
 
 size_t tree_smem(int D, int M0, int C) {
-    // 1 KB alignment, six [128 x D] images, 16 x 128 words of tables, 12 mbarriers,
-    // 4 words, the child counts of one (b,h)
-    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 16 + 12 * 8 + 16 + (size_t)M0 * C * 4;
+    // 1 KB alignment, six [128 x D] images, 16 x 128 words of tables, the
+    // mbarriers, 4 words, the child counts of one (b,h)
+    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 16 + kBars * 8 + 16 + (size_t)M0 * C * 4;
 }
 
 template <int D, int C>
