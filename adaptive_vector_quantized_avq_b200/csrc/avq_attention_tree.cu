@@ -237,7 +237,9 @@ __device__ __forceinline__ void select_top_p4(const float* part, unsigned long l
     }
 }
 
-template <int D, int C, int MINB>
+// FULL: 128 parents, so that each thread's parent blocks number four (fixed
+// loop counts)
+template <int D, int C, int MINB, bool FULL>
 __global__ void __launch_bounds__(kThreads, MINB)
 attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                       const __grid_constant__ CUtensorMap tmCB, const __grid_constant__ CUtensorMap tmMN,
@@ -357,14 +359,67 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     int cur_bh = -1;
     bool mma1_chained = false;   // (leader) this tile's MMA1 went out at the end of the previous tile
     const float2 sl2v = make_float2(p.sl2, p.sl2);
+    bool ok = true;
+    // ---- epilogue of tile (et, ebh): O = Xbar / Zbar -> bf16 -> swizzled
+    // staging -> TMA store (this thread: output dimensions hf * OD .. + OD - 1).
+    // It runs one tile late, after the next tile's first parent pass, so that
+    // the tile's last contraction completes under that pass. True when a wait
+    // gave up (for every thread).
+    auto epilogue = [&](int et, int ebh, float eden) -> bool {
+        sZ[hf * 128 + r] = eden;
+        ok = wait_bar(bO, oph, sAbort) && ok;
+        oph ^= 1;
+        tc_fence_after();
+        uint32_t packed[OD / 2];
+        {
+            float o[OD];
+#pragma unroll
+            for (int c = 0; c < OD / 16; ++c) tmem_ld16f(trow + p.colO + hf * OD + 16 * c, o + 16 * c);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < OD / 16; ++c) tmem_touch16f(o + 16 * c);
+            tc_fence_before();
+            pair_sync(q);
+            const float inv = 1.f / (sZ[r] + sZ[128 + r]);
+            const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+            for (int i = 0; i < OD / 2; ++i) {
+                const float2 v2 = fmul2(make_float2(o[2 * i], o[2 * i + 1]), inv2);
+                packed[i] = pack_bf16x2(v2.x, v2.y);
+            }
+        }
+        if (PC == 0 && store_thread) bulk_wait_read_all();
+        if (wg_sync_or(!ok)) return true;   // (and: the staging buffer is free)
+#pragma unroll
+        for (int j = 0; j < OD / 8; ++j)
+            *reinterpret_cast<uint4*>(sMC + swz(r, hf * (OD / 8) + j)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        fence_proxy_async_smem();
+        wg_sync();
+        if (store_thread) {
+#pragma unroll
+            for (int kh = 0; kh < KH; ++kh) tma_store_3d(&tmO, sMC + kh * kRegion, kh * 64, et * kTile, ebh);
+            bulk_commit();
+        }
+        return false;
+    };
+    bool pend = false;   // a tile whose epilogue is still to run
+    int pend_t = 0, pend_bh = 0;
+    float pend_den = 0.f;
     if (leader && g0 < g1) issue_q(g0, 0);
     for (int g = g0, it = 0; g < g1; ++g, ++it) {
         const int stage = it & 1;
         const int bh = g / p.ntiles, t = g % p.ntiles, h = bh % p.H;
+        // the next tile's MMA1 goes out with this tile's last contraction when it
+        // uses the same parent tables
+        const bool chain_next = g + 1 < g1 && (g + 1) / p.ntiles == bh;
         const int rows = min(kTile, p.N - t * kTile);
         const bool valid = r < rows;
-        bool ok = true;
         if (bh != cur_bh) {   // this (b,h)'s parent tables, log-counts and child counts
+            if (pend) {       // the previous tile's output first (its contractions end there)
+                if (epilogue(pend_t, pend_bh, pend_den)) { failed = true; break; }
+                pend = false;
+            }
             wg_sync();        // (every thread is past the previous tile, whose contractions are done)
             if (leader) {     // parent codewords and parent means (TMA)
                 head_pending = true;
@@ -412,8 +467,9 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         // Zbar (exact) and the denominator of the rounded weights. Two
         // passes over S_p (the shift, then the weights), one block at a time.
         float m, den;
+        bool epi_failed = false;
         {
-            const int nbp = (p.M0p / 16 + 1 - hf) / 2;   // this thread's parent blocks
+            const int nbp = FULL ? 4 : (p.M0p / 16 + 1 - hf) / 2;   // this thread's parent blocks
             float mp0 = -INFINITY, mp1 = -INFINITY;
             for (int i = 0; i < nbp; ++i) {
                 const int b = 2 * i + hf;
@@ -433,6 +489,14 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             sX[hf * 128 + r] = fmaxf(mp0, mp1);
             pair_sync(q);
             m = fmaxf(sX[r], sX[128 + r]);
+            if (pend) {   // the previous tile's output (its last contraction ran under the pass above)
+                epi_failed = epilogue(pend_t, pend_bh, pend_den);
+                pend = false;
+            }
+        }
+        if (epi_failed) { failed = true; break; }
+        {
+            const int nbp = FULL ? 4 : (p.M0p / 16 + 1 - hf) / 2;
             const float2 negm = make_float2(-m, -m);
             float2 z0 = make_float2(0.f, 0.f), z1 = make_float2(0.f, 0.f);
             float2 zb0 = make_float2(0.f, 0.f), zb1 = make_float2(0.f, 0.f);
@@ -490,7 +554,7 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int b = 2 * i + hf;
-                        if (16 * b < p.M0p) {
+                        if (FULL || 16 * b < p.M0p) {
                             tmem_ld_16x256b_x2(tmem + ((uint32_t)(32 * q + 16 * hh) << 16) + 16 * b, e + 8 * i);
                         } else {
 #pragma unroll
@@ -723,7 +787,7 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                     }
                     for (int i = 0; i < 4; ++i) {         // this thread's blocks of W_p
                         const int b = 2 * i + hf;
-                        if (16 * b >= p.M0p) break;
+                        if (!FULL && 16 * b >= p.M0p) break;
                         uint32_t u[8];
                         tmem_ld8(trow + p.colWp + 8 * b, u);
                         tmem_wait_ld();
@@ -751,6 +815,12 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                 if (wg_sync_or(!ok)) { failed = true; break; }
                 if (leader) {   // MMA3c O += W_c x mean_child (the last chunk's W_c is over W_p)
                     tc_fence_after();
+                    // after the last chunk every S column of this tile has been read
+                    // and no contraction left reads one: the next tile's MMA1 first
+                    if (k + 1 == nchunks && chain_next) {
+                        if (issue_mma1(g + 1, stage ^ 1)) mma1_chained = true;
+                        else ok = false;   // (seen by everyone at the next barrier)
+                    }
                     for (int ks = 0; ks < N2 / 16; ++ks)
                         mma_ts(tmem + p.colO, tmem + colWc + 8 * ks, desc_mn(sMC, ks), idesc3, 1);
                     mma_commit(k + 1 < nchunks ? bC : bO);
@@ -762,59 +832,22 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             if (wg_sync_or(!ok)) { failed = true; break; }
             if (leader) {   // MMA3p O = W_p x mean_par, the tile's only value contraction
                 tc_fence_after();
+                if (chain_next) {   // (S_p is read: the next tile's MMA1 first)
+                    if (issue_mma1(g + 1, stage ^ 1)) mma1_chained = true;
+                    else ok = false;
+                }
                 for (int ks = 0; ks < p.M0p / 16; ++ks)
                     mma_ts(tmem + p.colO, tmem + p.colWp + 8 * ks, desc_mn(sMP, ks), idesc3, ks > 0);
                 mma_commit(bO);
             }
             __syncwarp();
         }
-        // the next tile's MMA1 follows this tile's last contraction when it uses
-        // the same parent tables (every S column of this tile has been read, and
-        // no contraction above reads one)
-        if (leader && g + 1 < g1 && (g + 1) / p.ntiles == bh) {
-            if (issue_mma1(g + 1, stage ^ 1)) mma1_chained = true;
-            else ok = false;   // (seen by everyone at the barrier below)
-        }
-        __syncwarp();
-
-        // ---- epilogue: O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store
-        // (this thread: output dimensions hf * OD .. hf * OD + OD - 1)
-        sZ[hf * 128 + r] = den;
-        ok = wait_bar(bO, oph, sAbort) && ok;
-        oph ^= 1;
-        tc_fence_after();
-        uint32_t packed[OD / 2];
-        {
-            float o[OD];
-#pragma unroll
-            for (int c = 0; c < OD / 16; ++c) tmem_ld16f(trow + p.colO + hf * OD + 16 * c, o + 16 * c);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < OD / 16; ++c) tmem_touch16f(o + 16 * c);
-            tc_fence_before();
-            pair_sync(q);
-            const float inv = 1.f / (sZ[r] + sZ[128 + r]);
-            const float2 inv2 = make_float2(inv, inv);
-#pragma unroll
-            for (int i = 0; i < OD / 2; ++i) {
-                const float2 v2 = fmul2(make_float2(o[2 * i], o[2 * i + 1]), inv2);
-                packed[i] = pack_bf16x2(v2.x, v2.y);
-            }
-        }
-        if (PC == 0 && store_thread) bulk_wait_read_all();
-        if (wg_sync_or(!ok)) { failed = true; break; }   // the staging buffer is free
-#pragma unroll
-        for (int j = 0; j < OD / 8; ++j)
-            *reinterpret_cast<uint4*>(sMC + swz(r, hf * (OD / 8) + j)) =
-                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-        fence_proxy_async_smem();
-        wg_sync();
-        if (store_thread) {
-#pragma unroll
-            for (int kh = 0; kh < KH; ++kh) tma_store_3d(&tmO, sMC + kh * kRegion, kh * 64, t * kTile, bh);
-            bulk_commit();
-        }
+        pend = true;
+        pend_t = t;
+        pend_bh = bh;
+        pend_den = den;
     }
+    if (!failed && pend && epilogue(pend_t, pend_bh, pend_den)) failed = true;
     cp_async_wait_all();
     if (store_thread) bulk_wait_all();
 
@@ -880,7 +913,8 @@ cudaError_t launch_tree(const avq_shape& s, const void* Q, const void* cb, const
     prm.status = status;
     prm.fail_first_wait = g_fail_next_wait.exchange(0);
     const size_t smem = tree_smem(D, s.M0, C);
-    auto kern = attention_tree_kernel<D, C, MINB>;
+    const bool full = M0p == 128;
+    auto kern = full ? attention_tree_kernel<D, C, MINB, true> : attention_tree_kernel<D, C, MINB, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
