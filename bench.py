@@ -595,7 +595,8 @@ def run_reference(args):
     }), flush=True)
 
 
-KERNEL_NAMES = {"precompute": "precompute_tc_kernel", "attention": "attention_tc_kernel"}
+KERNEL_NAMES = {"precompute": ("precompute_tc_kernel", "flat_precompute_kernel", "deep_precompute_kernel"),
+                "attention": ("attention_tree_kernel", "flat_attention_kernel", "deep_attention_kernel")}
 
 
 def ingest_ncu(csv_path: str, workload: str, P: int):
@@ -619,7 +620,7 @@ def ingest_ncu(csv_path: str, workload: str, P: int):
         per[(d["ID"], name)][metric] = float(val.replace(",", "")) * scale
     out = json.load(open(PROFILE_TRAFFIC)) if os.path.exists(PROFILE_TRAFFIC) else {}
     for kind, kname in KERNEL_NAMES.items():
-        launches = [m for (i, n), m in per.items() if kname in n and "dram__bytes_read.sum" in m]
+        launches = [m for (i, n), m in per.items() if any(k in n for k in kname) and "dram__bytes_read.sum" in m]
         if not launches:
             continue
         b = [m["dram__bytes_read.sum"] + m.get("dram__bytes_write.sum", 0.0) for m in launches]
