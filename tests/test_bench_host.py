@@ -47,7 +47,7 @@ def test_ingest_records_traffic_per_launch(tmp_path, monkeypatch):
             '"Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"\n')
     rows = []
     for i, (name, rd, wr) in enumerate([("void avq::precompute_tc_kernel<64, 8, 4>(x)", "200.0", "4.0"),
-                                        ("void avq::attention_tc_kernel<64, 8, 2>(x)", "100.0", "50.0"),
+                                        ("void avq::attention_tree_kernel<64, 8, 2, true>(x)", "100.0", "50.0"),
                                         ("void avq::precompute_tc_kernel<64, 8, 4>(x)", "202.0", "4.0")]):
         for metric, unit, val in (("dram__bytes_read.sum", "Mbyte", rd), ("dram__bytes_write.sum", "Mbyte", wr)):
             rows.append(f'"{i}","1","python","h","{name}","1","7","(1,1,1)","(1,1,1)","0","10.0",'
