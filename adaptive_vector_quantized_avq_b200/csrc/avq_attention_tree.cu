@@ -266,7 +266,10 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     float* sZ = sX + 256;                    // [2][128] row exchange: Zbar, then the denominator
     float* sT = sZ + 256;                    // [2][128] row exchange: largest child exponent
     int* sSel = reinterpret_cast<int*>(sT + 256);              // [128] selected parents by rank
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + 128);
+    // [128] per selected parent: its W_p column (offset from colWp), and the
+    // bits of 1 / n_p with the sign bit set when its weight is the low bf16 half
+    uint2* sLk = reinterpret_cast<uint2*>(sSel + 128);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sLk + 128);
     uint64_t* bQ = bars;                     // [2] Q stage landed
     uint64_t* bHead = bars + 2;              // head tables landed
     uint64_t* bS = bars + 3;                 // MMA1 / MMA2 done (S_p, S_c ready)
@@ -605,6 +608,11 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             if (store_thread) bulk_wait_read_all();   // the previous O store has read the staging
             wg_sync();   // the selection is in sSel
             gat_pending = tma_gather;   // (leader: the gather below is in flight until bGatT completes)
+            if (ct < p.P) {   // where the child pass finds each selected parent's weight
+                const int pid = min(max(sSel[ct], 0), p.M0 - 1);
+                sLk[ct] = make_uint2((uint32_t)(pid >> 1),
+                                     __float_as_uint(sInvN[pid]) | ((pid & 1) ? 0u : 0x80000000u));
+            }
             {
                 if (tma_gather) {   // each selected parent's children: one TMA load per image
                     // (slot s from thread 32 (s % 8) + s / 8: the loads leave from all
@@ -728,20 +736,21 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                         float sc[16];
                         float nap[PB];
                         {
-                            int pid[PB];
-                            uint32_t wr[PB];
+                            uint32_t wr[PB], code[PB];
                             tmem_ld16f(trow + 16 * b, sc);
 #pragma unroll
-                            for (int j = 0; j < PB; ++j) {
-                                pid[j] = min(max(sSel[min((cs + 16 * b) / C + j, p.P - 1)], 0), p.M0 - 1);
-                                tmem_ld1(trow + p.colWp + (pid[j] >> 1), wr[j]);
+                            for (int j = 0; j < PB; ++j) {   // -A_p = -W_p / n_p of the block's parents
+                                const uint2 lk = sLk[min((cs + 16 * b) / C + j, p.P - 1)];
+                                code[j] = lk.y;
+                                tmem_ld1(trow + p.colWp + lk.x, wr[j]);
                             }
                             tmem_wait_ld();
                             tmem_touch16f(sc);
 #pragma unroll
                             for (int j = 0; j < PB; ++j) {
                                 tmem_touch1(wr[j]);
-                                nap[j] = -((pid[j] & 1) ? bf16_hi(wr[j]) : bf16_lo(wr[j])) * sInvN[pid[j]];
+                                const uint32_t w = (wr[j] << ((code[j] >> 27) & 16u)) & 0xFFFF0000u;
+                                nap[j] = __uint_as_float(code[j] | 0x80000000u) * __uint_as_float(w);
                             }
                         }
 #pragma unroll
@@ -874,9 +883,9 @@ attention_tree_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 }
 
 size_t tree_smem(int D, int M0, int C) {
-    // 1 KB alignment, six [128 x D] images, 16 x 128 words of tables, the
+    // 1 KB alignment, six [128 x D] images, 18 x 128 words of tables, the
     // mbarriers, 4 words, the child counts of one (b,h)
-    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 16 + kBars * 8 + 16 + (size_t)M0 * C * 4;
+    return 1024 + 6 * (size_t)(D / 64) * kRegion + 128 * 4 * 18 + kBars * 8 + 16 + (size_t)M0 * C * 4;
 }
 
 template <int D, int C>
