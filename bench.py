@@ -119,14 +119,23 @@ def roofline_for(kind, alg, ms, peaks, sustained):
             "roofline_us": t_hbm * 1e6}
 
 
-def kernel_source_hash(kind: str) -> str:
-    """Hash of the sources a kernel is built from (to invalidate stored ncu traffic)."""
+# the sources the two calls' kernels are built from (tree, flat and depth-L
+# paths, with the shared headers and the entry points); other kernels of the
+# library do not change their traffic
+KERNEL_SOURCES = ("avq_api.cu", "avq_internal.cuh", "avq_sm100.cuh", "avq_tma.cu", "avq_precompute_tc.cu",
+                  "avq_attention_tree.cu", "avq_attention_tc.cu", "avq_deep.cu")
+
+
+def kernel_source_hash(kind: str, deep: bool = False) -> str:
+    """Hash of the sources a call's kernels are built from (to invalidate stored
+    ncu traffic): the depth-L kernels for a deeper tree, else the others."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "adaptive_vector_quantized_avq_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(n.encode() + f.read())
+    shared = ("avq_api.cu", "avq_internal.cuh", "avq_sm100.cuh")
+    names = shared + (("avq_deep.cu",) if deep else tuple(n for n in KERNEL_SOURCES if n not in shared + ("avq_deep.cu",)))
+    for n in sorted(names):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -138,7 +147,7 @@ def stored_traffic(kind: str, workload: str, P: int):
     with open(PROFILE_TRAFFIC) as f:
         d = json.load(f)
     e = d.get(f"{kind}/{workload}/P{P}")
-    if not e or e.get("source_hash") != kernel_source_hash(kind):
+    if not e or e.get("source_hash") != kernel_source_hash(kind, syn.WORKLOADS[workload].L > 2):
         return None
     return e.get("bytes_per_launch")
 
@@ -626,7 +635,7 @@ def ingest_ncu(csv_path: str, workload: str, P: int):
         b = [m["dram__bytes_read.sum"] + m.get("dram__bytes_write.sum", 0.0) for m in launches]
         out[f"{kind}/{workload}/P{P}"] = {
             "bytes_per_launch": sum(b) / len(b), "launches": len(b),
-            "source_hash": kernel_source_hash(kind), "from": os.path.basename(csv_path)}
+            "source_hash": kernel_source_hash(kind, syn.WORKLOADS[workload].L > 2), "from": os.path.basename(csv_path)}
     os.makedirs(os.path.dirname(PROFILE_TRAFFIC), exist_ok=True)
     with open(PROFILE_TRAFFIC, "w") as f:
         json.dump(out, f, indent=1, sort_keys=True)
