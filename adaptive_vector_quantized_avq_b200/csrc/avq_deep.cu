@@ -21,8 +21,8 @@
 //     P_l largest are expanded (ties to the lower row id), and every child g
 //     of an expanded node f adds (A_g - A_f) [vsum_g, n_g] to Xbar and Zbar.
 //
-// Both kernels run on CUDA cores. The precompute takes one warp per key and
-// decides every comparison on exact fp64 distances summed in index order,
+// Both kernels run on CUDA cores. The precompute takes one thread per key
+// and decides every comparison on exact fp64 distances summed in index order,
 // so its decisions are the exact ones by construction. The attention takes
 // one CTA per query tile (one thread per row) with the row's Xbar in
 // registers and the per-candidate weights in shared memory.
@@ -67,49 +67,78 @@ long long deep_rows(int M0, int C, int L) {
     return acc;
 }
 
-// lexicographic (distance, index) minimum over the warp
-__device__ __forceinline__ void warp_argmin(double& d, int& i) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        const double od = __shfl_xor_sync(0xffffffffu, d, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-        if (od < d || (od == d && oi < i)) {
-            d = od;
-            i = oi;
-        }
-    }
-}
-
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
 
-// One warp per key: lanes split the candidates of each step; every distance
-// is exact_sq_dist (fp64, index order, no fusion). The key's path nodes
-// count it and sum its value row (16-byte vector reductions, lanes over d).
+// element e (0 .. 4 / sizeof(T) - 1) of a 32-bit word of T values, as fp64
+// (exact: bf16 and fp32 values widen without rounding)
+__device__ __forceinline__ double word_elem(uint32_t w, int e, const __nv_bfloat16*) {
+    return (double)__uint_as_float(e == 0 ? w << 16 : w & 0xFFFF0000u);
+}
+__device__ __forceinline__ double word_elem(uint32_t w, int, const float*) { return (double)__uint_as_float(w); }
+
+// One thread per key (a block: 128 keys of one (b,h)). The head's level-0
+// rows are staged in shared memory (every thread of a warp reads the same
+// row at the same time: broadcasts), the key row is held in registers, and
+// the deeper levels' candidate rows are read with 16-byte loads. Every
+// distance is the fp64 sum of squared differences in index order without
+// fusion, exactly as exact_sq_dist forms it, and candidates are scanned in
+// index order with a strict comparison: the decisions are the exact ones.
+// The key's path nodes count it and sum its value row (16-byte vector
+// reductions).
 template <typename T, int D>
-__global__ void __launch_bounds__(256)
-deep_precompute_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ cb,
-                       int32_t* __restrict__ assign, int32_t* __restrict__ counts, float* __restrict__ vsum,
-                       long long R, int N, int H, DeepTree t) {
-    const long long key = (long long)(((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-    const int lane = threadIdx.x & 31;
-    if (key >= R) return;
-    const long long bh = key / N;
-    const int h = (int)(bh % H);
-    const T* k = K + key * D;
+__global__ void __launch_bounds__(128)
+deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ cb,
+                            int32_t* __restrict__ assign, int32_t* __restrict__ counts, float* __restrict__ vsum,
+                            int N, int H, int ntiles, DeepTree t) {
+    constexpr int W = D * (int)sizeof(T) / 4;   // 32-bit words per row
+    constexpr int EPW = 4 / (int)sizeof(T);     // elements per word
+    constexpr int U = W / 4;                    // 16-byte chunks per row
+    extern __shared__ uint4 sC4[];              // [M0][U] the head's level-0 rows
+    const int bh = blockIdx.x / ntiles, tile = blockIdx.x % ntiles, h = bh % H;
     const T* cbh = cb + (size_t)h * t.Mtot * D;
+    for (int i = threadIdx.x; i < t.M0 * U; i += blockDim.x) sC4[i] = __ldg(reinterpret_cast<const uint4*>(cbh) + i);
+    __syncthreads();
+    const int n = tile * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    const size_t key = (size_t)bh * N + n;
+    uint32_t kw[W];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(K + key * D) + j);
+        kw[4 * j] = u.x;
+        kw[4 * j + 1] = u.y;
+        kw[4 * j + 2] = u.z;
+        kw[4 * j + 3] = u.w;
+    }
+    const T* tag = nullptr;
+    auto dist = [&](const uint4* row, bool shared) -> double {
+        double acc = 0.0;
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const uint4 u = shared ? row[j] : __ldg(row + j);
+            const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+                for (int e = 0; e < EPW; ++e) {
+                    const double tt = __dsub_rn(word_elem(kw[4 * j + w], e, tag), word_elem(cw[w], e, tag));
+                    acc = __dadd_rn(acc, __dmul_rn(tt, tt));
+                }
+        }
+        return acc;
+    };
     double best = INFINITY;
     int bi = t.M0;
-    for (int q = lane; q < t.M0; q += 32) {
-        const double s = exact_sq_dist(k, cbh + (size_t)q * D, D);
-        if (s < best) {
-            best = s;
+    for (int q = 0; q < t.M0; ++q) {
+        const double dq = dist(sC4 + (size_t)q * U, true);
+        if (dq < best) {
+            best = dq;
             bi = q;
         }
     }
-    warp_argmin(best, bi);
     int local = bi < t.M0 ? bi : 0;   // (only non-finite inputs leave bi == M0)
     int node = local;
     int path[kMaxL];
@@ -118,14 +147,13 @@ deep_precompute_kernel(const T* __restrict__ K, const T* __restrict__ V, const T
     for (int l = 1; l < t.L; ++l) {
         double dc = INFINITY;
         int ci = t.C;
-        for (int c = lane; c < t.C; c += 32) {
-            const double s = exact_sq_dist(k, cbh + (size_t)(t.off[l] + local * t.C + c) * D, D);
-            if (s < dc) {
-                dc = s;
+        for (int c = 0; c < t.C; ++c) {
+            const double dq = dist(reinterpret_cast<const uint4*>(cbh + (size_t)(t.off[l] + local * t.C + c) * D), false);
+            if (dq < dc) {
+                dc = dq;
                 ci = c;
             }
         }
-        warp_argmin(dc, ci);
         if (!(ci < t.C && dc < best)) break;   // no child strictly closer: the descent stops
         best = dc;
         local = local * t.C + ci;
@@ -133,15 +161,23 @@ deep_precompute_kernel(const T* __restrict__ K, const T* __restrict__ V, const T
         path[depth++] = node;
     }
     const size_t base = (size_t)bh * t.Mtot;
-    if (lane == 0) {
-        assign[key] = node;
-        for (int i = 0; i < depth; ++i) atomicAdd(counts + base + path[i], 1);
-    }
-    // value row: lane j4 takes elements 4 j4 .. 4 j4 + 3
-    for (int j4 = lane; j4 < D / 4; j4 += 32) {
-        const float a = ld_f32(V + key * D + 4 * j4), b = ld_f32(V + key * D + 4 * j4 + 1);
-        const float c = ld_f32(V + key * D + 4 * j4 + 2), e = ld_f32(V + key * D + 4 * j4 + 3);
-        for (int i = 0; i < depth; ++i) red_add_v4(vsum + (base + path[i]) * D + 4 * j4, a, b, c, e);
+    assign[key] = node;
+    for (int i = 0; i < depth; ++i) atomicAdd(counts + base + path[i], 1);
+    // value row: four elements per reduction, for every node on the path
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(V + key * D) + j);
+        const uint32_t vw[4] = {u.x, u.y, u.z, u.w};
+        float f[4 * EPW];
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+            for (int e = 0; e < EPW; ++e) f[w * EPW + e] = (float)word_elem(vw[w], e, tag);
+#pragma unroll
+        for (int g = 0; g < EPW; ++g)
+            for (int i = 0; i < depth; ++i)
+                red_add_v4(vsum + (base + path[i]) * D + (size_t)j * 4 * EPW + 4 * g, f[4 * g], f[4 * g + 1],
+                           f[4 * g + 2], f[4 * g + 3]);
     }
 }
 
@@ -336,11 +372,14 @@ size_t deep_attn_smem(int D, int KT) {
 template <typename T, int D>
 cudaError_t launch_deep_pre(const avq_shape& s, const DeepTree& t, const void* K, const void* V, const void* cb,
                             int32_t* assign, int32_t* counts, float* vsum, cudaStream_t st) {
-    const long long R = (long long)s.B * s.H * s.N;
-    const long long blocks = (R * 32 + 255) / 256;
-    deep_precompute_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
-        static_cast<const T*>(K), static_cast<const T*>(V), static_cast<const T*>(cb), assign, counts, vsum, R, s.N,
-        s.H, t);
+    const int ntiles = (s.N + 127) / 128;
+    const size_t smem = (size_t)t.M0 * D * sizeof(T);
+    auto kern = deep_precompute_rows_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)((long long)s.B * s.H * ntiles), 128, smem, st>>>(
+        static_cast<const T*>(K), static_cast<const T*>(V), static_cast<const T*>(cb), assign, counts, vsum, s.N, s.H,
+        ntiles, t);
     count_launch();
     return cudaGetLastError();
 }
