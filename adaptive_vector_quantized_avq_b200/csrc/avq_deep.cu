@@ -208,14 +208,14 @@ struct DeepAttnArgs {
 // memory (padded strides keep both the per-row and the per-candidate access
 // patterns free of bank conflicts):
 //   Qs   [D][KT]            the tile's queries as fp32, transposed
-//   E    [kCand][KT + 1]    e'_c = A_c n_c of the current candidates per row
-//   Ap   [kCand][KT + 1]    A_f of the expanded candidates (by rank) per row
-//   W    [kCand]            importance of the current candidates
-//   cid  [kCand]            candidate row ids;  par [kCand]: rank of a
-//                           candidate's expanded parent;  sel [kCand]: the
+//   E    [KC][KT + 1]       e'_c = A_c n_c of the current candidates per row
+//   Ap   [KC][KT + 1]       A_f of the expanded candidates (by rank) per row
+//   W    [KC]               importance of the current candidates
+//   cid  [KC]               candidate row ids;  par [KC]: rank of a
+//                           candidate's expanded parent;  sel [KC]: the
 //                           expanded candidates (indices) by rank
-//   Zs   [KT]               Zbar per row (0 for rows past the end)
-template <typename T, int D, int KT>
+//   Zs   [KT]               1 / Zbar per row (0 for rows past the end)
+template <typename T, int D, int KT, int KC>
 __global__ void __launch_bounds__(KT)
 deep_attention_kernel(const DeepAttnArgs a) {
     extern __shared__ float sm[];
@@ -226,13 +226,13 @@ deep_attention_kernel(const DeepAttnArgs a) {
     const int i = tt * KT + r;
     const bool valid = i < a.N;
     float* Qs = sm;                                  // [D][KT]
-    float* E = Qs + D * KT;                          // [kCand][ES]
-    float* Ap = E + kCand * ES;                      // [kCand][ES]
-    float* W = Ap + kCand * ES;                      // [kCand]
-    float* Zs = W + kCand;                           // [KT]
-    int* cid = reinterpret_cast<int*>(Zs + KT);      // [kCand]
-    int* par = cid + kCand;                          // [kCand]
-    int* sel = par + kCand;                          // [kCand]
+    float* E = Qs + D * KT;                          // [KC][ES]
+    float* Ap = E + KC * ES;                         // [KC][ES]
+    float* W = Ap + KC * ES;                         // [KC]
+    float* Zs = W + KC;                              // [KT]
+    int* cid = reinterpret_cast<int*>(Zs + KT);      // [KC]
+    int* par = cid + KC;                             // [KC]
+    int* sel = par + KC;                             // [KC]
     const T* Q = static_cast<const T*>(a.Q);
     const T* cbh = static_cast<const T*>(a.cb) + (size_t)h * t.Mtot * D;
     const int32_t* cnt = a.counts + (size_t)bh * t.Mtot;
@@ -245,15 +245,37 @@ deep_attention_kernel(const DeepAttnArgs a) {
         Qs[j * KT + rr] = ii < a.N ? ld_f32(Q + ((size_t)bh * a.N + ii) * D + j) : 0.f;
     }
     __syncthreads();
-    auto logit = [&](int row) -> float {   // Q_i . codeword(row), fp32
-        const T* c = cbh + (size_t)row * D;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < D; j += 2) {
-            s0 = fmaf(Qs[j * KT + r], ld_f32(c + j), s0);
-            s1 = fmaf(Qs[(j + 1) * KT + r], ld_f32(c + j + 1), s1);
+    // Q_i . codeword(row), fp32, in four interleaved sums (the row read 16
+    // bytes at a time: every thread of the CTA reads the same row)
+    auto logit = [&](int row) -> float {
+        constexpr int EPV = 16 / (int)sizeof(T);   // elements per 16 bytes
+        constexpr int EPW = 4 / (int)sizeof(T);    // elements per 32-bit word
+        const uint4* c4 = reinterpret_cast<const uint4*>(cbh + (size_t)row * D);
+        const T* tag = nullptr;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};   // element j goes to sum j % 4
+#pragma unroll 2
+        for (int v = 0; v < D / EPV; ++v) {
+            const uint4 u = __ldg(c4 + v);
+            const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) {
+                const int j = v * EPV + e;
+                s4[j % 4] = fmaf(Qs[j * KT + r], (float)word_elem(cw[e / EPW], e % EPW, tag), s4[j % 4]);
+            }
         }
-        return s0 + s1;
+        return (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    };
+    // x += w * mean(row), the mean row read 16 bytes at a time
+    auto add_mean = [&](float (&xx)[D], float w, int row) {
+        const float4* m4 = reinterpret_cast<const float4*>(mn + (size_t)row * D);
+#pragma unroll
+        for (int v = 0; v < D / 4; ++v) {
+            const float4 q4 = __ldg(m4 + v);
+            xx[4 * v] = fmaf(w, q4.x, xx[4 * v]);
+            xx[4 * v + 1] = fmaf(w, q4.y, xx[4 * v + 1]);
+            xx[4 * v + 2] = fmaf(w, q4.z, xx[4 * v + 2]);
+            xx[4 * v + 3] = fmaf(w, q4.w, xx[4 * v + 3]);
+        }
     };
 
     float x[D];
@@ -273,23 +295,23 @@ deep_attention_kernel(const DeepAttnArgs a) {
         const float e = exp2f(E[c * ES + r] - m);   // 0 for empty nodes
         E[c * ES + r] = e;
         z += e;
-        const float* mc = mn + (size_t)c * D;
-#pragma unroll
-        for (int j = 0; j < D; ++j) x[j] = fmaf(e, __ldg(mc + j), x[j]);
+        add_mean(x, e, c);
     }
     for (int c = r; c < ncand; c += KT) cid[c] = c;
     int soff = 0;
     for (int l = 0; l + 1 < t.L; ++l) {
-        Zs[r] = valid ? z : 0.f;
+        Zs[r] = valid && z > 0.f ? 1.f / z : 0.f;
         __syncthreads();
-        // importance: sum over the tile's rows of e' / Zbar (Zbar so far)
+        // importance: sum over the tile's rows of e' / Zbar (Zbar so far), as
+        // e' times the row's 1 / Zbar (0 for rows past the end)
         for (int c = r; c < ncand; c += KT) {
-            float w = 0.f;
-            for (int rr = 0; rr < KT; ++rr) {
-                const float zz = Zs[rr];
-                if (zz > 0.f) w += E[c * ES + rr] / zz;
+            float w0 = 0.f, w1 = 0.f;
+#pragma unroll 4
+            for (int rr = 0; rr < KT; rr += 2) {
+                w0 = fmaf(E[c * ES + rr], Zs[rr], w0);
+                w1 = fmaf(E[c * ES + rr + 1], Zs[rr + 1], w1);
             }
-            W[c] = w;
+            W[c] = w0 + w1;
         }
         __syncthreads();
         const int P = min(a.P[l], ncand);
@@ -314,7 +336,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
         }
         __syncthreads();   // every row has read the expanded candidates' ids and weights
         // the next candidates: the children of the expanded ones, in rank order
-        int nid[kCand / 32 + 1];
+        int nid[KC / 32 + 1];
         int nn = 0;
         for (int s = r; s < P * t.C; s += KT) nid[nn++] = t.off[l + 1] + (cid[sel[s / t.C]] - t.off[l]) * t.C + s % t.C;
         __syncthreads();
@@ -348,9 +370,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
                 e = exp2f(u);
                 const float dw = e - Ap[par[c] * ES + r] * (float)n;   // (A_g - A_f) n_g
                 z += dw;
-                const float* mc = mn + (size_t)row * D;
-#pragma unroll
-                for (int j = 0; j < D; ++j) x[j] = fmaf(dw, __ldg(mc + j), x[j]);
+                add_mean(x, dw, row);
             }
             E[c * ES + r] = e;
         }
@@ -365,8 +385,8 @@ deep_attention_kernel(const DeepAttnArgs a) {
     }
 }
 
-size_t deep_attn_smem(int D, int KT) {
-    return sizeof(float) * ((size_t)D * KT + 2 * (size_t)kCand * (KT + 1) + kCand + KT) + sizeof(int) * 3 * kCand;
+size_t deep_attn_smem(int D, int KT, int KC) {
+    return sizeof(float) * ((size_t)D * KT + 2 * (size_t)KC * (KT + 1) + KC + KT) + sizeof(int) * 3 * KC;
 }
 
 template <typename T, int D>
@@ -384,10 +404,10 @@ cudaError_t launch_deep_pre(const avq_shape& s, const DeepTree& t, const void* K
     return cudaGetLastError();
 }
 
-template <typename T, int D, int KT>
+template <typename T, int D, int KT, int KC>
 cudaError_t launch_deep_att(const DeepAttnArgs& a, int tiles, cudaStream_t st) {
-    const size_t smem = deep_attn_smem(D, KT);
-    auto kern = deep_attention_kernel<T, D, KT>;
+    const size_t smem = deep_attn_smem(D, KT, KC);
+    auto kern = deep_attention_kernel<T, D, KT, KC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)tiles, KT, smem, st>>>(a);
@@ -488,8 +508,15 @@ int avq_attention_deep(const avq_shape* s, int L, const int32_t* P, const void* 
     a.sl2 = scale * 1.4426950408889634f;
     const int tiles = s->B * s->H * a.ntiles;
     cudaError_t e;
-#define AVQ_DEEP_CASE(TT, DD, KK) \
-    if (s->d == DD && tile == KK) e = launch_deep_att<TT, DD, KK>(a, tiles, st);
+    // candidates per level held on chip: 64 when no level has more (the
+    // per-row tables halve: two CTAs per SM at d = 64 and 128-row tiles),
+    // else 128
+    int maxc = s->M0;
+    for (int l = 0; l + 1 < L; ++l) maxc = std::max(maxc, a.P[l] * s->C);
+    const bool kc64 = maxc <= 64;
+#define AVQ_DEEP_CASE(TT, DD, KK)                                                                     \
+    if (s->d == DD && tile == KK)                                                                     \
+        e = kc64 ? launch_deep_att<TT, DD, KK, 64>(a, tiles, st) : launch_deep_att<TT, DD, KK, 128>(a, tiles, st);
     if (s->dtype == AVQ_BF16) {
         AVQ_DEEP_CASE(__nv_bfloat16, 64, 64) AVQ_DEEP_CASE(__nv_bfloat16, 64, 128)
         AVQ_DEEP_CASE(__nv_bfloat16, 128, 64) AVQ_DEEP_CASE(__nv_bfloat16, 128, 128)
