@@ -215,7 +215,14 @@ struct DeepAttnArgs {
 //                           candidate's expanded parent;  sel [KC]: the
 //                           expanded candidates (indices) by rank
 //   Zs   [KT]               1 / Zbar per row (0 for rows past the end)
-template <typename T, int D, int KT, int KC>
+//   ncs  [KC]               counts of the current candidates
+//   Cw   [KC][D]            the current candidates' codewords (raw T rows)
+//   Mn   [KC][D]            their value means (fp32)
+// At d = 64 the row's query is held in registers instead of Qs. With ST the
+// candidates' rows are staged once per level (Cw, Mn), so that the
+// per-candidate loop reads shared-memory broadcasts; without (when they would
+// not fit) it reads them from global memory, 16 bytes at a time.
+template <typename T, int D, int KT, int KC, bool ST>
 __global__ void __launch_bounds__(KT)
 deep_attention_kernel(const DeepAttnArgs a) {
     extern __shared__ float sm[];
@@ -225,52 +232,80 @@ deep_attention_kernel(const DeepAttnArgs a) {
     const int r = threadIdx.x;
     const int i = tt * KT + r;
     const bool valid = i < a.N;
-    float* Qs = sm;                                  // [D][KT]
-    float* E = Qs + D * KT;                          // [KC][ES]
+    constexpr bool QREG = D <= 64;                   // the query row in registers
+    constexpr int CU = D * (int)sizeof(T) / 16;      // 16-byte chunks of a codeword row
+    constexpr int MU = D / 4;                        // 16-byte chunks of a mean row
+    float* Qs = sm;                                  // [D][KT] (unless QREG)
+    float* E = Qs + (QREG ? 0 : D * KT);             // [KC][ES]
     float* Ap = E + KC * ES;                         // [KC][ES]
     float* W = Ap + KC * ES;                         // [KC]
     float* Zs = W + KC;                              // [KT]
     int* cid = reinterpret_cast<int*>(Zs + KT);      // [KC]
     int* par = cid + KC;                             // [KC]
     int* sel = par + KC;                             // [KC]
+    int* ncs = sel + KC;                             // [KC]
+    uint4* Cw = reinterpret_cast<uint4*>(ncs + KC);  // [KC][CU] (16-byte aligned: every array above is a multiple of 4 words)
+    float4* Mn = reinterpret_cast<float4*>(Cw + KC * CU);   // [KC][MU]
     const T* Q = static_cast<const T*>(a.Q);
     const T* cbh = static_cast<const T*>(a.cb) + (size_t)h * t.Mtot * D;
     const int32_t* cnt = a.counts + (size_t)bh * t.Mtot;
     const float* mn = a.mean + (size_t)bh * t.Mtot * D;
 
-    // the tile's queries, transposed (coalesced reads of whole rows)
-    for (int idx = r; idx < KT * D; idx += KT) {
-        const int rr = idx / D, j = idx % D;
-        const int ii = tt * KT + rr;
-        Qs[j * KT + rr] = ii < a.N ? ld_f32(Q + ((size_t)bh * a.N + ii) * D + j) : 0.f;
+    const T* tag = nullptr;
+    constexpr int EPV = 16 / (int)sizeof(T);   // elements per 16 bytes
+    constexpr int EPW = 4 / (int)sizeof(T);    // elements per 32-bit word
+    float qv[QREG ? D : 1];
+    if constexpr (QREG) {   // this row's query
+        const uint4* q4 = reinterpret_cast<const uint4*>(Q + ((size_t)bh * a.N + (valid ? i : 0)) * D);
+#pragma unroll
+        for (int v = 0; v < CU; ++v) {
+            const uint4 u = valid ? __ldg(q4 + v) : make_uint4(0, 0, 0, 0);
+            const uint32_t qw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) qv[v * EPV + e] = (float)word_elem(qw[e / EPW], e % EPW, tag);
+        }
+    } else {   // the tile's queries, transposed (coalesced reads of whole rows)
+        for (int idx = r; idx < KT * D; idx += KT) {
+            const int rr = idx / D, j = idx % D;
+            const int ii = tt * KT + rr;
+            Qs[j * KT + rr] = ii < a.N ? ld_f32(Q + ((size_t)bh * a.N + ii) * D + j) : 0.f;
+        }
     }
-    __syncthreads();
-    // Q_i . codeword(row), fp32, in four interleaved sums (the row read 16
-    // bytes at a time: every thread of the CTA reads the same row)
-    auto logit = [&](int row) -> float {
-        constexpr int EPV = 16 / (int)sizeof(T);   // elements per 16 bytes
-        constexpr int EPW = 4 / (int)sizeof(T);    // elements per 32-bit word
-        const uint4* c4 = reinterpret_cast<const uint4*>(cbh + (size_t)row * D);
-        const T* tag = nullptr;
+    // the nc current candidates' rows (ids in cid), counts, codewords and
+    // value means, into shared memory (every thread; ends at a CTA barrier)
+    auto stage = [&](int nc) {
+        if constexpr (ST) {
+            for (int idx = r; idx < nc * CU; idx += KT)
+                Cw[idx] = __ldg(reinterpret_cast<const uint4*>(cbh + (size_t)cid[idx / CU] * D) + idx % CU);
+            for (int idx = r; idx < nc * MU; idx += KT)
+                Mn[idx] = __ldg(reinterpret_cast<const float4*>(mn + (size_t)cid[idx / MU] * D) + idx % MU);
+        }
+        for (int c = r; c < nc; c += KT) ncs[c] = __ldg(cnt + cid[c]);
+        __syncthreads();
+    };
+    // Q_i . codeword of candidate slot sl, fp32, in four interleaved sums
+    auto logit = [&](int sl) -> float {
+        const uint4* c4 = ST ? Cw + sl * CU : reinterpret_cast<const uint4*>(cbh + (size_t)cid[sl] * D);
         float s4[4] = {0.f, 0.f, 0.f, 0.f};   // element j goes to sum j % 4
-#pragma unroll 2
-        for (int v = 0; v < D / EPV; ++v) {
-            const uint4 u = __ldg(c4 + v);
+#pragma unroll
+        for (int v = 0; v < CU; ++v) {
+            const uint4 u = ST ? c4[v] : __ldg(c4 + v);
             const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int e = 0; e < EPV; ++e) {
                 const int j = v * EPV + e;
-                s4[j % 4] = fmaf(Qs[j * KT + r], (float)word_elem(cw[e / EPW], e % EPW, tag), s4[j % 4]);
+                const float qj = QREG ? qv[QREG ? j : 0] : Qs[j * KT + r];
+                s4[j % 4] = fmaf(qj, (float)word_elem(cw[e / EPW], e % EPW, tag), s4[j % 4]);
             }
         }
         return (s4[0] + s4[1]) + (s4[2] + s4[3]);
     };
-    // x += w * mean(row), the mean row read 16 bytes at a time
-    auto add_mean = [&](float (&xx)[D], float w, int row) {
-        const float4* m4 = reinterpret_cast<const float4*>(mn + (size_t)row * D);
+    // x += w * the value mean of candidate slot sl
+    auto add_mean = [&](float (&xx)[D], float w, int sl) {
+        const float4* m4 = ST ? Mn + sl * MU : reinterpret_cast<const float4*>(mn + (size_t)cid[sl] * D);
 #pragma unroll
         for (int v = 0; v < D / 4; ++v) {
-            const float4 q4 = __ldg(m4 + v);
+            const float4 q4 = ST ? m4[v] : __ldg(m4 + v);
             xx[4 * v] = fmaf(w, q4.x, xx[4 * v]);
             xx[4 * v + 1] = fmaf(w, q4.y, xx[4 * v + 1]);
             xx[4 * v + 2] = fmaf(w, q4.z, xx[4 * v + 2]);
@@ -283,9 +318,12 @@ deep_attention_kernel(const DeepAttnArgs a) {
     for (int j = 0; j < D; ++j) x[j] = 0.f;
     // level 0: log-count logits, the row's shift m, weights e' = 2^(x - m)
     int ncand = t.M0;
+    for (int c = r; c < ncand; c += KT) cid[c] = c;
+    __syncthreads();
+    stage(ncand);
     float m = -INFINITY;
     for (int c = 0; c < ncand; ++c) {
-        const int n = __ldg(cnt + c);
+        const int n = ncs[c];
         const float xv = n > 0 ? fmaf(logit(c), a.sl2, __log2f((float)n)) : -INFINITY;
         E[c * ES + r] = xv;
         m = fmaxf(m, xv);
@@ -297,7 +335,6 @@ deep_attention_kernel(const DeepAttnArgs a) {
         z += e;
         add_mean(x, e, c);
     }
-    for (int c = r; c < ncand; c += KT) cid[c] = c;
     int soff = 0;
     for (int l = 0; l + 1 < t.L; ++l) {
         Zs[r] = valid && z > 0.f ? 1.f / z : 0.f;
@@ -331,7 +368,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
         // candidates are replaced by their children
         for (int k = 0; k < P; ++k) {
             const int c = sel[k];
-            const int n = __ldg(cnt + cid[c]);
+            const int n = ncs[c];
             Ap[k * ES + r] = n > 0 ? E[c * ES + r] / (float)n : 0.f;
         }
         __syncthreads();   // every row has read the expanded candidates' ids and weights
@@ -347,12 +384,12 @@ deep_attention_kernel(const DeepAttnArgs a) {
         }
         __syncthreads();
         ncand = P * t.C;
+        stage(ncand);
         for (int c = 0; c < ncand; ++c) {
-            const int row = cid[c];
-            const int n = __ldg(cnt + row);
+            const int n = ncs[c];
             float e = 0.f;
             if (n > 0) {
-                float u = fmaf(logit(row), a.sl2, __log2f((float)n)) - m;
+                float u = fmaf(logit(c), a.sl2, __log2f((float)n)) - m;
                 if (u > kRescale) {
                     // a child far above the row's shift: move the shift up by a
                     // whole number k of octaves and scale everything this row
@@ -370,7 +407,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
                 e = exp2f(u);
                 const float dw = e - Ap[par[c] * ES + r] * (float)n;   // (A_g - A_f) n_g
                 z += dw;
-                add_mean(x, dw, row);
+                add_mean(x, dw, c);
             }
             E[c * ES + r] = e;
         }
@@ -385,8 +422,10 @@ deep_attention_kernel(const DeepAttnArgs a) {
     }
 }
 
-size_t deep_attn_smem(int D, int KT, int KC) {
-    return sizeof(float) * ((size_t)D * KT + 2 * (size_t)KC * (KT + 1) + KC + KT) + sizeof(int) * 3 * KC;
+size_t deep_attn_smem(int D, int KT, int KC, size_t elem, bool staged) {
+    const size_t qs = D <= 64 ? 0 : (size_t)D * KT;   // (the query rows are in registers at d <= 64)
+    return sizeof(float) * (qs + 2 * (size_t)KC * (KT + 1) + KC + KT) + sizeof(int) * 4 * KC +
+           (staged ? (size_t)KC * D * (elem + sizeof(float)) : 0);
 }
 
 template <typename T, int D>
@@ -406,8 +445,10 @@ cudaError_t launch_deep_pre(const avq_shape& s, const DeepTree& t, const void* K
 
 template <typename T, int D, int KT, int KC>
 cudaError_t launch_deep_att(const DeepAttnArgs& a, int tiles, cudaStream_t st) {
-    const size_t smem = deep_attn_smem(D, KT, KC);
-    auto kern = deep_attention_kernel<T, D, KT, KC>;
+    // the candidates' rows staged in shared memory when the CTA still fits
+    const bool staged = deep_attn_smem(D, KT, KC, sizeof(T), true) <= 227 * 1024;
+    const size_t smem = deep_attn_smem(D, KT, KC, sizeof(T), staged);
+    auto kern = staged ? deep_attention_kernel<T, D, KT, KC, true> : deep_attention_kernel<T, D, KT, KC, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)tiles, KT, smem, st>>>(a);
