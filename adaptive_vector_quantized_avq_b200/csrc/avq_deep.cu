@@ -322,6 +322,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
     __syncthreads();
     stage(ncand);
     float m = -INFINITY;
+#pragma unroll 2
     for (int c = 0; c < ncand; ++c) {
         const int n = ncs[c];
         const float xv = n > 0 ? fmaf(logit(c), a.sl2, __log2f((float)n)) : -INFINITY;
@@ -329,6 +330,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
         m = fmaxf(m, xv);
     }
     float z = 0.f;
+#pragma unroll 2
     for (int c = 0; c < ncand; ++c) {
         const float e = exp2f(E[c * ES + r] - m);   // 0 for empty nodes
         E[c * ES + r] = e;
@@ -385,26 +387,37 @@ deep_attention_kernel(const DeepAttnArgs a) {
         __syncthreads();
         ncand = P * t.C;
         stage(ncand);
+        // pass 1: every candidate's exponent u = sl2 S + log2 n - m and the
+        // largest one (the candidates are independent: unrolled for overlap)
+        float umax = -INFINITY;
+#pragma unroll 2
+        for (int c = 0; c < ncand; ++c) {
+            const int n = ncs[c];
+            const float u = n > 0 ? fmaf(logit(c), a.sl2, __log2f((float)n)) - m : -INFINITY;
+            E[c * ES + r] = u;
+            umax = fmaxf(umax, u);
+        }
+        float ku = 0.f;
+        if (umax > kRescale) {
+            // a child far above the row's shift: move the shift up by a whole
+            // number k of octaves and scale everything this row holds by 2^-k
+            // (exact), so that no weight overflows
+            ku = ceilf(umax);
+            const float f = exp2f(-ku);
+            m += ku;
+            z *= f;
+#pragma unroll
+            for (int j = 0; j < D; ++j) x[j] *= f;
+            for (int kk = 0; kk < P; ++kk) Ap[kk * ES + r] *= f;
+        }
+        // pass 2: weights e' = 2^u, the corrections (A_g - A_f) n_g into Zbar
+        // and Xbar
+#pragma unroll 2
         for (int c = 0; c < ncand; ++c) {
             const int n = ncs[c];
             float e = 0.f;
             if (n > 0) {
-                float u = fmaf(logit(c), a.sl2, __log2f((float)n)) - m;
-                if (u > kRescale) {
-                    // a child far above the row's shift: move the shift up by a
-                    // whole number k of octaves and scale everything this row
-                    // holds by 2^-k (exact), so that no weight overflows
-                    const float k = ceilf(u);
-                    const float f = exp2f(-k);
-                    m += k;
-                    u -= k;
-                    z *= f;
-#pragma unroll
-                    for (int j = 0; j < D; ++j) x[j] *= f;
-                    for (int cc = 0; cc < c; ++cc) E[cc * ES + r] *= f;
-                    for (int kk = 0; kk < P; ++kk) Ap[kk * ES + r] *= f;
-                }
-                e = exp2f(u);
+                e = exp2f(E[c * ES + r] - ku);
                 const float dw = e - Ap[par[c] * ES + r] * (float)n;   // (A_g - A_f) n_g
                 z += dw;
                 add_mean(x, dw, c);
