@@ -1,14 +1,15 @@
 // avq_attention_tree.cu -- tensor-core (tcgen05) kernel of avq_attention for
 // bf16 trees, 128-query tiles (paper §4.3; papernotes, Key Designs 3).
 //
-// Warp-specialised and persistent. A CTA has 288 threads: warp 0 issues the
-// loads of Q and of the head's parent tables (TMA) and every tcgen05.mma;
-// warps 1-8 compute, two threads per query row (warps w and w + 4 share the
-// TMEM lanes of the row; each takes every other 16-column block of the
-// parents, of the child slots and half of the output dimensions). The two
-// sides hand work over through mbarriers, so each contraction is issued the
-// moment its inputs are ready and the next tile's S = Q C^T runs under the
-// current tile's epilogue. Two CTAs share an SM at d = 64.
+// Persistent. A CTA has 256 threads, two per query row (warps w and w + 4
+// share the TMEM lanes of the row; each takes every other 16-column block of
+// the parents, of the child slots and half of the output dimensions). Thread
+// 0 also issues the loads of Q and of the head's parent tables (TMA) and
+// every tcgen05.mma, each right after the CTA barrier that already orders
+// its inputs; mbarriers carry only the tensor core's and TMA's completions.
+// The next tile's S = Q C^T is issued ahead of the current tile's last value
+// contraction, and each tile's epilogue runs one tile late, under the next
+// tile's first parent pass. Two CTAs share an SM at d = 64.
 //
 // TMEM (columns; 256 at d = 64, 512 at d = 128):
 //   [0, 128)          S_p = Q C_par^T (fp32); then e'_p (fp32) for the
@@ -29,20 +30,22 @@
 // contractions multiply (each weight rounded once, then used on both
 // sides). Per tile:
 //   1. MMA1 S_p; parent pass: x_p, m, e'_p, Zbar (fp32, exact, for the
-//      importance), bf16 W_p -> TMEM; MMA3p O = W_p x mean_par.
+//      importance), bf16 W_p -> TMEM; MMA3p O = W_p x mean_par (issued once
+//      every thread's W_p is written).
 //   2. Importance w_p = sum_rows e'_p / Zbar, from TMEM in the 16x256b
 //      layout (each thread holds four rows), a three-level butterfly and a
 //      four-warp sum in shared memory; top-P over 64-bit values (the bit
 //      pattern of w >= 0 above the complement of the index: ties to the lower
 //      index), each of four warps sorting 32 of them, a value's rank found
 //      by binary searches in the other warps' lists.
-//   3. Per chunk of <= 128 selected child slots: the compute threads gather
-//      the children's codewords and value means (cp.async), the producer
-//      issues MMA2 S_c; the child weight (A_c - A_p) n_c = 2^(x_c - m) -
+//   3. Per chunk of <= 128 selected child slots: the children's codewords and
+//      value means are gathered (TMA, else cp.async), thread 0 issues MMA2
+//      S_c; the child weight (A_c - A_p) n_c = 2^(x_c - m) -
 //      A_p n_c (the ΔA replacement of the papernotes summary in
 //      count-weighted form, A_p taken from the bf16 W_p that MMA3p used) ->
 //      bf16 W_c; MMA3c.
-//   4. O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store.
+//   4. O = Xbar / Zbar -> bf16 -> swizzled staging -> TMA store (one tile
+//      late).
 // A child logit far above the row's shift (more than 64 octaves) moves the
 // shift: the row's O, W_p, denominator and written child weights are scaled
 // by an exact power of two (paper §4.3: the running accumulators are
@@ -56,7 +59,7 @@
 namespace avq {
 
 // (test hook, see avq_test_fail_next_wait) the next tree attention launch gives
-// up its producer's first wait at once
+// up thread 0's first wait at once
 std::atomic<int> g_fail_next_wait{0};
 
 cudaError_t launch_means_bf16(const float* vsum, const int32_t* counts, void* means, size_t nrows, int d,
@@ -80,7 +83,7 @@ struct TreeParams {
     const uint16_t* means;       // [BH, Mtot, D] bf16 value means
     int32_t* selected;           // [BH, ntiles, P]
     StatusBlock* status;
-    int fail_first_wait;         // (test hook) the producer's first wait gives up at once
+    int fail_first_wait;         // (test hook) thread 0's first wait gives up at once
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {

@@ -306,8 +306,9 @@ int avq_device_status(void* workspace, void* stream);
 /*
  * Test hook for the failure path (no counterpart in the paper). The next
  * avq_attention call that runs the bf16 tensor-core tree kernel behaves as if
- * one of its bounded device-side waits had run out: its first wait on the
- * compute threads' first hand-over gets a limit of zero. Every CTA then stops
+ * one of its bounded device-side waits had run out: the first wait of each
+ * CTA's issuing thread (for its head's parent tables) gets a limit of zero.
+ * Every CTA then stops
  * at once: the loads and contractions it has in flight complete, its tensor
  * memory is freed, and the call reports AVQ_ETIMEOUT through
  * avq_device_status (its outputs are not meaningful). Later calls are
