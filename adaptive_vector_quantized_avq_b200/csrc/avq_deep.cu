@@ -22,8 +22,9 @@
 //     of an expanded node f adds (A_g - A_f) [vsum_g, n_g] to Xbar and Zbar.
 //
 // Both kernels run on CUDA cores. The precompute takes one thread per key
-// and decides every comparison on exact fp64 distances summed in index order,
-// so its decisions are the exact ones by construction. The attention takes
+// and decides every comparison on fp32 distances, again on exact fp64 ones
+// (summed in index order) wherever the fp32 error bound cannot, so its
+// decisions are the exact ones. The attention takes
 // one CTA per query tile (one thread per row) with the row's Xbar in
 // registers and the per-candidate weights in shared memory.
 #include <algorithm>
@@ -80,22 +81,23 @@ __device__ __forceinline__ double word_elem(uint32_t w, int e, const __nv_bfloat
 __device__ __forceinline__ double word_elem(uint32_t w, int, const float*) { return (double)__uint_as_float(w); }
 
 // One thread per key (a block: 128 keys of one (b,h)). The head's level-0
-// rows are staged in shared memory (every thread of a warp reads the same
-// row at the same time: broadcasts), the key row is held in registers, and
-// the deeper levels' candidate rows are read with 16-byte loads. Every
-// distance is the fp64 sum of squared differences in index order without
-// fusion, exactly as exact_sq_dist forms it, and candidates are scanned in
-// index order with a strict comparison: the decisions are the exact ones.
-// The key's path nodes count it and sum its value row (16-byte vector
-// reductions).
+// rows are staged in shared memory (every thread of a warp reads the same row
+// at the same time: broadcasts) and the key row is held in registers. Each
+// step is decided on fp32 squared distances (sum of fma(t, t) over t =
+// fl(k - c), whose error is bounded by dist_eps); where the bound cannot
+// separate the winner from another candidate, the step is decided again on
+// exact fp64 distances (exact_sq_dist: index order, no fusion) among the
+// candidates it cannot separate, so that every decision is the exact one:
+// level 0 the nearest node (first on ties), deeper levels a child only when
+// strictly closer than the current node (first child on ties). The key's
+// path nodes count it and sum its value row (16-byte vector reductions).
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
 deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ cb,
                             int32_t* __restrict__ assign, int32_t* __restrict__ counts, float* __restrict__ vsum,
                             int N, int H, int ntiles, DeepTree t) {
-    constexpr int W = D * (int)sizeof(T) / 4;   // 32-bit words per row
-    constexpr int EPW = 4 / (int)sizeof(T);     // elements per word
-    constexpr int U = W / 4;                    // 16-byte chunks per row
+    constexpr int EPW = 4 / (int)sizeof(T);     // elements per 32-bit word
+    constexpr int U = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
     extern __shared__ uint4 sC4[];              // [M0][U] the head's level-0 rows
     const int bh = blockIdx.x / ntiles, tile = blockIdx.x % ntiles, h = bh % H;
     const T* cbh = cb + (size_t)h * t.Mtot * D;
@@ -104,18 +106,20 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
     const int n = tile * blockDim.x + threadIdx.x;
     if (n >= N) return;
     const size_t key = (size_t)bh * N + n;
-    uint32_t kw[W];
+    const T* tag = nullptr;
+    float kf[D];   // the key row (exact in fp32)
 #pragma unroll
     for (int j = 0; j < U; ++j) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(K + key * D) + j);
-        kw[4 * j] = u.x;
-        kw[4 * j + 1] = u.y;
-        kw[4 * j + 2] = u.z;
-        kw[4 * j + 3] = u.w;
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+            for (int e = 0; e < EPW; ++e) kf[(4 * j + w) * EPW + e] = (float)word_elem(w4[w], e, tag);
     }
-    const T* tag = nullptr;
-    auto dist = [&](const uint4* row, bool shared) -> double {
-        double acc = 0.0;
+    // fp32 squared distance to a row (shared or global memory), in index order
+    auto dist32 = [&](const uint4* row, bool shared) -> float {
+        float acc = 0.f;
 #pragma unroll
         for (int j = 0; j < U; ++j) {
             const uint4 u = shared ? row[j] : __ldg(row + j);
@@ -124,20 +128,42 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
             for (int w = 0; w < 4; ++w)
 #pragma unroll
                 for (int e = 0; e < EPW; ++e) {
-                    const double tt = __dsub_rn(word_elem(kw[4 * j + w], e, tag), word_elem(cw[w], e, tag));
-                    acc = __dadd_rn(acc, __dmul_rn(tt, tt));
+                    const float tt = __fsub_rn(kf[(4 * j + w) * EPW + e], (float)word_elem(cw[w], e, tag));
+                    acc = __fmaf_rn(tt, tt, acc);
                 }
         }
         return acc;
     };
-    double best = INFINITY;
+    const float eps = dist_eps(D);
+    const T* krow = K + key * D;
+    auto row_of = [&](int r) { return reinterpret_cast<const uint4*>(cbh + (size_t)r * D); };
+    // level 0: the nearest node
+    float best = INFINITY, second = INFINITY;
     int bi = t.M0;
     for (int q = 0; q < t.M0; ++q) {
-        const double dq = dist(sC4 + (size_t)q * U, true);
+        const float dq = dist32(sC4 + (size_t)q * U, true);
         if (dq < best) {
+            second = best;
             best = dq;
             bi = q;
+        } else if (dq < second) {
+            second = dq;
         }
+    }
+    if (t.M0 > 1 && !separated(best, second, eps)) {   // exact, among those the bound cannot separate
+        double eb = INFINITY;
+        int ep = -1;
+        for (int q = 0; q < t.M0; ++q) {
+            const float dq = dist32(sC4 + (size_t)q * U, true);
+            if (separated(best, dq, eps)) continue;
+            const double e = exact_sq_dist(krow, cbh + (size_t)q * D, D);
+            if (e < eb) {
+                eb = e;
+                ep = q;
+            }
+        }
+        if (ep >= 0) bi = ep;   // (ep < 0 only for non-finite inputs)
+        best = dist32(sC4 + (size_t)(bi < t.M0 ? bi : 0) * U, true);
     }
     int local = bi < t.M0 ? bi : 0;   // (only non-finite inputs leave bi == M0)
     int node = local;
@@ -145,19 +171,39 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
     int depth = 1;
     path[0] = node;
     for (int l = 1; l < t.L; ++l) {
-        double dc = INFINITY;
-        int ci = t.C;
+        const int first = t.off[l] + local * t.C;
+        // the current node first, then its children in index order; a child
+        // wins only when strictly closer
+        float lo = best;
+        int ci = -1;
         for (int c = 0; c < t.C; ++c) {
-            const double dq = dist(reinterpret_cast<const uint4*>(cbh + (size_t)(t.off[l] + local * t.C + c) * D), false);
-            if (dq < dc) {
-                dc = dq;
+            const float dq = dist32(row_of(first + c), false);
+            if (dq < lo) {
+                lo = dq;
                 ci = c;
             }
         }
-        if (!(ci < t.C && dc < best)) break;   // no child strictly closer: the descent stops
-        best = dc;
+        bool sure = ci < 0 || separated(lo, best, eps);
+        for (int c = 0; c < t.C && sure; ++c)
+            if (c != ci && !separated(lo, dist32(row_of(first + c), false), eps)) sure = false;
+        if (!sure) {   // exact, among the node and the children the bound cannot separate from the winner
+            double eb = exact_sq_dist(krow, cbh + (size_t)node * D, D);
+            int win = -1;
+            for (int c = 0; c < t.C; ++c) {
+                if (separated(lo, dist32(row_of(first + c), false), eps)) continue;
+                const double e = exact_sq_dist(krow, cbh + (size_t)(first + c) * D, D);
+                if (e < eb) {
+                    eb = e;
+                    win = c;
+                }
+            }
+            ci = win;
+            if (ci >= 0) lo = dist32(row_of(first + ci), false);
+        }
+        if (ci < 0) break;   // no child strictly closer: the descent stops
+        best = lo;
         local = local * t.C + ci;
-        node = t.off[l] + local;
+        node = first + ci;
         path[depth++] = node;
     }
     const size_t base = (size_t)bh * t.Mtot;
