@@ -607,7 +607,7 @@ int avq_attention_deep(const avq_shape* s, int L, const int32_t* P, const void* 
     a.ntiles = (s->N + tile - 1) / tile;
     a.sl2 = scale * 1.4426950408889634f;
     const int tiles = s->B * s->H * a.ntiles;
-    cudaError_t e;
+    cudaError_t e = cudaErrorInvalidValue;   // (every supported d and tile has a case below)
     // candidates per level held on chip: 64 when no level has more (the
     // per-row tables halve: two CTAs per SM at d = 64 and 128-row tiles),
     // else 128
