@@ -281,8 +281,9 @@ int avq_gather_rows(const avq_shape* s, const void* src, void* dst, const int32_
  * tile level 0's expanded row ids by rank, then level 1's, ...
  *
  * Supported: 2 <= L <= 4, 1 <= M0 <= 128, C >= 1, d in {64, 128}, fp32 or
- * bf16, tile in {64, 128}. Both calls run on CUDA cores (fp64 distances;
- * fp32 attention). The attention workspace (fp32 value means and the status
+ * bf16, tile in {64, 128}. Both calls run on CUDA cores (fp32 distances,
+ * with exact fp64 ones wherever the fp32 error bound cannot decide; fp32
+ * attention). The attention workspace (fp32 value means and the status
  * word) is avq_attention_deep_workspace_bytes(s, L) bytes, 256-byte
  * aligned. Errors: AVQ_EINVAL (arguments), AVQ_EUNSUPPORTED (sizes),
  * AVQ_EWORKSPACE, AVQ_ECUDA. Neither call synchronises.
