@@ -89,3 +89,25 @@ def test_oracle_sample_is_bounded():
 def test_warmup_below_three_is_refused():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_traffic_hash_follows_each_path_sources(tmp_path, monkeypatch):
+    """A stored traffic figure is tied to the sources its kernels are built
+    from: editing the depth-L kernels leaves the tree path's figure valid and
+    the reverse."""
+    import shutil
+    csrc = os.path.join(ROOT, "adaptive_vector_quantized_avq_b200", "csrc")
+    fake = tmp_path / "repo"
+    shutil.copytree(csrc, fake / "adaptive_vector_quantized_avq_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(fake))
+    tree0, deep0 = bench.kernel_source_hash("attention"), bench.kernel_source_hash("attention", True)
+    assert tree0 != deep0
+    with open(fake / "adaptive_vector_quantized_avq_b200" / "csrc" / "avq_deep.cu", "a") as f:
+        f.write("\n// edit\n")
+    assert bench.kernel_source_hash("attention") == tree0
+    deep1 = bench.kernel_source_hash("attention", True)
+    assert deep1 != deep0
+    with open(fake / "adaptive_vector_quantized_avq_b200" / "csrc" / "avq_attention_tree.cu", "a") as f:
+        f.write("\n// edit\n")
+    assert bench.kernel_source_hash("attention") != tree0
+    assert bench.kernel_source_hash("attention", True) == deep1
