@@ -80,11 +80,43 @@ __device__ __forceinline__ double word_elem(uint32_t w, int e, const __nv_bfloat
 }
 __device__ __forceinline__ double word_elem(uint32_t w, int, const float*) { return (double)__uint_as_float(w); }
 
+// acc + a_h * b_h for the bf16 values in the low (h = 0) / high (h = 1) halves
+// of a and b: sm_100's mixed-precision fma, one rounding (the bf16 product is
+// exact in fp32, so this equals fmaf on the widened values)
+__device__ __forceinline__ float fma_bf16_lo(uint32_t a, uint32_t b, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}" : "=f"(r) : "r"(a), "r"(b), "f"(acc));
+    return r;
+}
+__device__ __forceinline__ float fma_bf16_hi(uint32_t a, uint32_t b, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}" : "=f"(r) : "r"(a), "r"(b), "f"(acc));
+    return r;
+}
+// k - c_h for the bf16 value c_h in the low / high half of w, rounded once
+// (the mixed-precision fma c_h * -1 + k; identical to __fsub_rn on the
+// widened value)
+__device__ __forceinline__ float sub_bf16_lo(float k, uint32_t w) {
+    float r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, l, %2, %3;\n\t}"
+        : "=f"(r) : "r"(w), "h"((unsigned short)0xBF80u), "f"(k));
+    return r;
+}
+__device__ __forceinline__ float sub_bf16_hi(float k, uint32_t w) {
+    float r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, h, %2, %3;\n\t}"
+        : "=f"(r) : "r"(w), "h"((unsigned short)0xBF80u), "f"(k));
+    return r;
+}
+
 // One thread per key (a block: 128 keys of one (b,h)). The head's level-0
 // rows are staged in shared memory (every thread of a warp reads the same row
 // at the same time: broadcasts) and the key row is held in registers. Each
-// step is decided on fp32 squared distances (sum of fma(t, t) over t =
-// fl(k - c), whose error is bounded by dist_eps); where the bound cannot
+// step is decided on fp32 squared distances (fma(t, t) over t = fl(k - c),
+// even and odd terms in two sums added at the end, whose error is bounded by
+// dist_eps); where the bound cannot
 // separate the winner from another candidate, the step is decided again on
 // exact fp64 distances (exact_sq_dist: index order, no fusion) among the
 // candidates it cannot separate, so that every decision is the exact one:
@@ -107,32 +139,48 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
     if (n >= N) return;
     const size_t key = (size_t)bh * N + n;
     const T* tag = nullptr;
-    float kf[D];   // the key row (exact in fp32)
+    // the key row, exact in fp32, as (even, odd) element pairs
+    float2 kf[D / 2];
 #pragma unroll
     for (int j = 0; j < U; ++j) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(K + key * D) + j);
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+        if constexpr (EPW == 2) {
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-#pragma unroll
-            for (int e = 0; e < EPW; ++e) kf[(4 * j + w) * EPW + e] = (float)word_elem(w4[w], e, tag);
+            for (int w = 0; w < 4; ++w)
+                kf[4 * j + w] = make_float2(__uint_as_float(w4[w] << 16), __uint_as_float(w4[w] & 0xFFFF0000u));
+        } else {
+            kf[2 * j] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+            kf[2 * j + 1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+        }
     }
-    // fp32 squared distance to a row (shared or global memory), in index order
+    // fp32 squared distance to a row (shared or global memory): t = fl(k - c)
+    // in one rounding, then fma(t, t) into an even-element and an odd-element
+    // sum (sm_100 paired fp32 fma), added at the end -- two chains of d/2
+    // terms, within the (d+2)u of dist_eps
     auto dist32 = [&](const uint4* row, bool shared) -> float {
-        float acc = 0.f;
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < U; ++j) {
             const uint4 u = shared ? row[j] : __ldg(row + j);
-            const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
+            if constexpr (EPW == 2) {
+                const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
-#pragma unroll
-                for (int e = 0; e < EPW; ++e) {
-                    const float tt = __fsub_rn(kf[(4 * j + w) * EPW + e], (float)word_elem(cw[w], e, tag));
-                    acc = __fmaf_rn(tt, tt, acc);
+                for (int w = 0; w < 4; ++w) {
+                    const float2 tt = make_float2(sub_bf16_lo(kf[4 * j + w].x, cw[w]),
+                                                  sub_bf16_hi(kf[4 * j + w].y, cw[w]));
+                    acc = __ffma2_rn(tt, tt, acc);
                 }
+            } else {
+                const float2 m1 = make_float2(-1.f, -1.f);
+                const float2 ta = __ffma2_rn(make_float2(__uint_as_float(u.x), __uint_as_float(u.y)), m1, kf[2 * j]);
+                const float2 tb =
+                    __ffma2_rn(make_float2(__uint_as_float(u.z), __uint_as_float(u.w)), m1, kf[2 * j + 1]);
+                acc = __ffma2_rn(ta, ta, acc);
+                acc = __ffma2_rn(tb, tb, acc);
+            }
         }
-        return acc;
+        return __fadd_rn(acc.x, acc.y);
     };
     const float eps = dist_eps(D);
     const T* krow = K + key * D;
@@ -245,6 +293,7 @@ struct DeepAttnArgs {
     void* O;
     int32_t* selected;     // [BH, ntiles, sum_l P_l], level after level
     int N, H, ntiles, Psum;
+    int ap_words;          // words of the Ap table: (largest P) rows of KT + 1, rounded up to 4
     int P[kMaxL];
     float sl2;             // scale * log2(e)
     DeepTree t;
@@ -255,8 +304,9 @@ struct DeepAttnArgs {
 // patterns free of bank conflicts):
 //   Qs   [D][KT]            the tile's queries as fp32, transposed
 //   E    [KC][KT + 1]       e'_c = A_c n_c of the current candidates per row
-//   Ap   [KC][KT + 1]       A_f of the expanded candidates (by rank) per row
+//   Ap   [Pmax][KT + 1]     A_f of the expanded candidates (by rank) per row
 //   W    [KC]               importance of the current candidates
+//   lgn  [KC]               log2 of the current candidates' counts
 //   cid  [KC]               candidate row ids;  par [KC]: rank of a
 //                           candidate's expanded parent;  sel [KC]: the
 //                           expanded candidates (indices) by rank
@@ -264,7 +314,8 @@ struct DeepAttnArgs {
 //   ncs  [KC]               counts of the current candidates
 //   Cw   [KC][D]            the current candidates' codewords (raw T rows)
 //   Mn   [KC][D]            their value means (fp32)
-// At d = 64 the row's query is held in registers instead of Qs. With ST the
+// At d = 64 the row's query is held in registers instead of Qs (bf16: packed,
+// its logits by mixed-precision fma on the packed words). With ST the
 // candidates' rows are staged once per level (Cw, Mn), so that the
 // per-candidate loop reads shared-memory broadcasts; without (when they would
 // not fit) it reads them from global memory, 16 bytes at a time.
@@ -283,10 +334,11 @@ deep_attention_kernel(const DeepAttnArgs a) {
     constexpr int MU = D / 4;                        // 16-byte chunks of a mean row
     float* Qs = sm;                                  // [D][KT] (unless QREG)
     float* E = Qs + (QREG ? 0 : D * KT);             // [KC][ES]
-    float* Ap = E + KC * ES;                         // [KC][ES]
-    float* W = Ap + KC * ES;                         // [KC]
+    float* Ap = E + KC * ES;                         // [Pmax][ES]
+    float* W = Ap + a.ap_words;                      // [KC]
     float* Zs = W + KC;                              // [KT]
-    int* cid = reinterpret_cast<int*>(Zs + KT);      // [KC]
+    float* lgn = Zs + KT;                            // [KC]
+    int* cid = reinterpret_cast<int*>(lgn + KC);     // [KC]
     int* par = cid + KC;                             // [KC]
     int* sel = par + KC;                             // [KC]
     int* ncs = sel + KC;                             // [KC]
@@ -300,15 +352,22 @@ deep_attention_kernel(const DeepAttnArgs a) {
     const T* tag = nullptr;
     constexpr int EPV = 16 / (int)sizeof(T);   // elements per 16 bytes
     constexpr int EPW = 4 / (int)sizeof(T);    // elements per 32-bit word
-    float qv[QREG ? D : 1];
+    constexpr bool QPK = QREG && EPW == 2;           // bf16 row kept packed, two values per word
+    float qv[(QREG && !QPK) ? D : 1];
+    uint32_t qp[QPK ? D / 2 : 1];
     if constexpr (QREG) {   // this row's query
         const uint4* q4 = reinterpret_cast<const uint4*>(Q + ((size_t)bh * a.N + (valid ? i : 0)) * D);
 #pragma unroll
         for (int v = 0; v < CU; ++v) {
             const uint4 u = valid ? __ldg(q4 + v) : make_uint4(0, 0, 0, 0);
             const uint32_t qw[4] = {u.x, u.y, u.z, u.w};
+            if constexpr (QPK) {
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) qv[v * EPV + e] = (float)word_elem(qw[e / EPW], e % EPW, tag);
+                for (int w = 0; w < 4; ++w) qp[QPK ? 4 * v + w : 0] = qw[w];
+            } else {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) qv[QPK ? 0 : v * EPV + e] = (float)word_elem(qw[e / EPW], e % EPW, tag);
+            }
         }
     } else {   // the tile's queries, transposed (coalesced reads of whole rows)
         for (int idx = r; idx < KT * D; idx += KT) {
@@ -326,7 +385,11 @@ deep_attention_kernel(const DeepAttnArgs a) {
             for (int idx = r; idx < nc * MU; idx += KT)
                 Mn[idx] = __ldg(reinterpret_cast<const float4*>(mn + (size_t)cid[idx / MU] * D) + idx % MU);
         }
-        for (int c = r; c < nc; c += KT) ncs[c] = __ldg(cnt + cid[c]);
+        for (int c = r; c < nc; c += KT) {
+            const int n = __ldg(cnt + cid[c]);
+            ncs[c] = n;
+            lgn[c] = n > 0 ? __log2f((float)n) : -INFINITY;
+        }
         __syncthreads();
     };
     // Q_i . codeword of candidate slot sl, fp32, in four interleaved sums
@@ -337,11 +400,19 @@ deep_attention_kernel(const DeepAttnArgs a) {
         for (int v = 0; v < CU; ++v) {
             const uint4 u = ST ? c4[v] : __ldg(c4 + v);
             const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
+            if constexpr (QPK) {   // element 8v + 2w + h is word w's half h
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) {
-                const int j = v * EPV + e;
-                const float qj = QREG ? qv[QREG ? j : 0] : Qs[j * KT + r];
-                s4[j % 4] = fmaf(qj, (float)word_elem(cw[e / EPW], e % EPW, tag), s4[j % 4]);
+                for (int w = 0; w < 4; ++w) {
+                    s4[(2 * w) % 4] = fma_bf16_lo(qp[QPK ? 4 * v + w : 0], cw[w], s4[(2 * w) % 4]);
+                    s4[(2 * w + 1) % 4] = fma_bf16_hi(qp[QPK ? 4 * v + w : 0], cw[w], s4[(2 * w + 1) % 4]);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) {
+                    const int j = v * EPV + e;
+                    const float qj = QREG ? qv[QREG ? j : 0] : Qs[j * KT + r];
+                    s4[j % 4] = fmaf(qj, (float)word_elem(cw[e / EPW], e % EPW, tag), s4[j % 4]);
+                }
             }
         }
         return (s4[0] + s4[1]) + (s4[2] + s4[3]);
@@ -371,7 +442,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
 #pragma unroll 2
     for (int c = 0; c < ncand; ++c) {
         const int n = ncs[c];
-        const float xv = n > 0 ? fmaf(logit(c), a.sl2, __log2f((float)n)) : -INFINITY;
+        const float xv = n > 0 ? fmaf(logit(c), a.sl2, lgn[c]) : -INFINITY;
         E[c * ES + r] = xv;
         m = fmaxf(m, xv);
     }
@@ -439,7 +510,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
 #pragma unroll 2
         for (int c = 0; c < ncand; ++c) {
             const int n = ncs[c];
-            const float u = n > 0 ? fmaf(logit(c), a.sl2, __log2f((float)n)) - m : -INFINITY;
+            const float u = n > 0 ? fmaf(logit(c), a.sl2, lgn[c]) - m : -INFINITY;
             E[c * ES + r] = u;
             umax = fmaxf(umax, u);
         }
@@ -481,9 +552,17 @@ deep_attention_kernel(const DeepAttnArgs a) {
     }
 }
 
-size_t deep_attn_smem(int D, int KT, int KC, size_t elem, bool staged) {
+// words of the Ap table: one row of KT + 1 per expanded candidate of the
+// level that expands the most, rounded up to 4 (keeps the arrays after it
+// 16-byte aligned)
+int deep_ap_words(const DeepAttnArgs& a, int KT) {
+    int pmax = 0;
+    for (int l = 0; l + 1 < a.t.L; ++l) pmax = std::max(pmax, a.P[l]);
+    return (pmax * (KT + 1) + 3) & ~3;
+}
+size_t deep_attn_smem(int D, int KT, int KC, size_t elem, bool staged, int ap_words) {
     const size_t qs = D <= 64 ? 0 : (size_t)D * KT;   // (the query rows are in registers at d <= 64)
-    return sizeof(float) * (qs + 2 * (size_t)KC * (KT + 1) + KC + KT) + sizeof(int) * 4 * KC +
+    return sizeof(float) * (qs + (size_t)KC * (KT + 1) + (size_t)ap_words + 2 * KC + KT) + sizeof(int) * 4 * KC +
            (staged ? (size_t)KC * D * (elem + sizeof(float)) : 0);
 }
 
@@ -503,10 +582,11 @@ cudaError_t launch_deep_pre(const avq_shape& s, const DeepTree& t, const void* K
 }
 
 template <typename T, int D, int KT, int KC>
-cudaError_t launch_deep_att(const DeepAttnArgs& a, int tiles, cudaStream_t st) {
+cudaError_t launch_deep_att(DeepAttnArgs a, int tiles, cudaStream_t st) {
+    a.ap_words = deep_ap_words(a, KT);
     // the candidates' rows staged in shared memory when the CTA still fits
-    const bool staged = deep_attn_smem(D, KT, KC, sizeof(T), true) <= 227 * 1024;
-    const size_t smem = deep_attn_smem(D, KT, KC, sizeof(T), staged);
+    const bool staged = deep_attn_smem(D, KT, KC, sizeof(T), true, a.ap_words) <= 227 * 1024;
+    const size_t smem = deep_attn_smem(D, KT, KC, sizeof(T), staged, a.ap_words);
     auto kern = staged ? deep_attention_kernel<T, D, KT, KC, true> : deep_attention_kernel<T, D, KT, KC, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
