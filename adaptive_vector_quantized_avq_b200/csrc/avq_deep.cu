@@ -37,6 +37,7 @@ namespace {
 constexpr int kMaxL = 4;       // levels of a tree (level 0 .. 3)
 constexpr int kCand = 128;     // candidates per level held on chip
 constexpr float kRescale = 64.f;   // largest weight exponent (log2) before a row's shift moves
+constexpr int kCh = 4;         // children per node whose distances the precompute keeps in registers
 
 struct DeepTree {
     int M0, C, L, Mtot;
@@ -122,7 +123,9 @@ __device__ __forceinline__ float sub_bf16_hi(float k, uint32_t w) {
 // candidates it cannot separate, so that every decision is the exact one:
 // level 0 the nearest node (first on ties), deeper levels a child only when
 // strictly closer than the current node (first child on ties). The key's
-// path nodes count it and sum its value row (16-byte vector reductions).
+// own node (the deepest on its path) counts it and sums its value row
+// (16-byte vector reductions; the row was prefetched to L2 at the start);
+// deep_totals_kernel then gives every node its whole subtree.
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
 deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ cb,
@@ -138,6 +141,11 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
     const int n = tile * blockDim.x + threadIdx.x;
     if (n >= N) return;
     const size_t key = (size_t)bh * N + n;
+    {   // the value row is read after the descent: start bringing it to L2 now
+        const char* vrow = reinterpret_cast<const char*>(V + key * D);
+#pragma unroll
+        for (int o = 0; o < D * (int)sizeof(T); o += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(vrow + o));
+    }
     const T* tag = nullptr;
     // the key row, exact in fp32, as (even, odd) element pairs
     float2 kf[D / 2];
@@ -215,16 +223,27 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
     }
     int local = bi < t.M0 ? bi : 0;   // (only non-finite inputs leave bi == M0)
     int node = local;
-    int path[kMaxL];
-    int depth = 1;
-    path[0] = node;
     for (int l = 1; l < t.L; ++l) {
         const int first = t.off[l] + local * t.C;
         // the current node first, then its children in index order; a child
         // wins only when strictly closer
+        // (the first kCh children's distances stay in registers for the
+        // separation test)
         float lo = best;
         int ci = -1;
-        for (int c = 0; c < t.C; ++c) {
+        float dch[kCh];
+#pragma unroll
+        for (int c = 0; c < kCh; ++c) {
+            dch[c] = INFINITY;
+            if (c < t.C) {
+                dch[c] = dist32(row_of(first + c), false);
+                if (dch[c] < lo) {
+                    lo = dch[c];
+                    ci = c;
+                }
+            }
+        }
+        for (int c = kCh; c < t.C; ++c) {
             const float dq = dist32(row_of(first + c), false);
             if (dq < lo) {
                 lo = dq;
@@ -232,7 +251,10 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
             }
         }
         bool sure = ci < 0 || separated(lo, best, eps);
-        for (int c = 0; c < t.C && sure; ++c)
+#pragma unroll
+        for (int c = 0; c < kCh; ++c)
+            if (c < t.C && c != ci && !separated(lo, dch[c], eps)) sure = false;
+        for (int c = kCh; c < t.C && sure; ++c)
             if (c != ci && !separated(lo, dist32(row_of(first + c), false), eps)) sure = false;
         if (!sure) {   // exact, among the node and the children the bound cannot separate from the winner
             double eb = exact_sq_dist(krow, cbh + (size_t)node * D, D);
@@ -252,12 +274,13 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
         best = lo;
         local = local * t.C + ci;
         node = first + ci;
-        path[depth++] = node;
     }
     const size_t base = (size_t)bh * t.Mtot;
     assign[key] = node;
-    for (int i = 0; i < depth; ++i) atomicAdd(counts + base + path[i], 1);
-    // value row: four elements per reduction, for every node on the path
+    // the key's count and value row go to its own node only (the deepest on
+    // its path); deep_totals_kernel then adds every node's subtree into it
+    atomicAdd(counts + base + node, 1);
+    // value row: four elements per reduction
 #pragma unroll
     for (int j = 0; j < U; ++j) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(V + key * D) + j);
@@ -269,9 +292,41 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
             for (int e = 0; e < EPW; ++e) f[w * EPW + e] = (float)word_elem(vw[w], e, tag);
 #pragma unroll
         for (int g = 0; g < EPW; ++g)
-            for (int i = 0; i < depth; ++i)
-                red_add_v4(vsum + (base + path[i]) * D + (size_t)j * 4 * EPW + 4 * g, f[4 * g], f[4 * g + 1],
-                           f[4 * g + 2], f[4 * g + 3]);
+            red_add_v4(vsum + (base + node) * D + (size_t)j * 4 * EPW + 4 * g, f[4 * g], f[4 * g + 1], f[4 * g + 2],
+                       f[4 * g + 3]);
+    }
+}
+
+// One level of the subtree totals, launched from the deepest level with
+// children upwards: each node of the level (width nodes from row `first`)
+// adds its C children's counts and value sums, complete by then, to those of
+// the keys that stopped at the node, so that it holds its whole subtree (the
+// "every node on a key's path counts the key" rule). One thread per (node,
+// 4 dimensions); the first of a node's threads also adds the counts.
+__global__ void deep_totals_kernel(int32_t* __restrict__ counts, float* __restrict__ vsum, size_t BH, int Mtot,
+                                   int first, int width, int child_first, int C, int d) {
+    const int q = d / 4;   // 16-byte chunks of a row
+    float4* v4 = reinterpret_cast<float4*>(vsum);
+    const size_t n = BH * (size_t)width * q;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n; idx += (size_t)gridDim.x * blockDim.x) {
+        const int k = (int)(idx % q);
+        const size_t nd = idx / q;
+        const int j = (int)(nd % width);
+        const size_t bh = nd / width;
+        const size_t row = bh * Mtot + first + j;
+        const size_t crow = bh * Mtot + child_first + (size_t)j * C;
+        float4 acc = v4[row * q + k];
+        int cn = 0;
+        for (int c = 0; c < C; ++c) {
+            const float4 v = v4[(crow + c) * q + k];
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+            if (k == 0) cn += counts[crow + c];
+        }
+        v4[row * q + k] = acc;
+        if (k == 0) counts[row] += cn;
     }
 }
 
@@ -578,7 +633,17 @@ cudaError_t launch_deep_pre(const avq_shape& s, const DeepTree& t, const void* K
         static_cast<const T*>(K), static_cast<const T*>(V), static_cast<const T*>(cb), assign, counts, vsum, s.N, s.H,
         ntiles, t);
     count_launch();
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t BH = (size_t)s.B * s.H;
+    for (int l = t.L - 2; l >= 0; --l) {
+        const int width = t.off[l + 1] - t.off[l];
+        const size_t n = BH * (size_t)width * (D / 4);
+        deep_totals_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, st>>>(
+            counts, vsum, BH, t.Mtot, t.off[l], width, t.off[l + 1], t.C, D);
+        count_launch();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 template <typename T, int D, int KT, int KC>
