@@ -373,9 +373,12 @@ struct DeepAttnArgs {
 // its logits by mixed-precision fma on the packed words). With ST the
 // candidates' rows are staged once per level (Cw, Mn), so that the
 // per-candidate loop reads shared-memory broadcasts; without (when they would
-// not fit) it reads them from global memory, 16 bytes at a time.
+// not fit) it reads them from global memory, 16 bytes at a time. The
+// candidate loops are unrolled four ways (more shared-memory reads in
+// flight); at d = 64 the launch bound keeps that within the registers of
+// three CTAs per SM.
 template <typename T, int D, int KT, int KC, bool ST>
-__global__ void __launch_bounds__(KT)
+__global__ void __launch_bounds__(KT, D == 64 ? 3 : 1)
 deep_attention_kernel(const DeepAttnArgs a) {
     extern __shared__ float sm[];
     constexpr int ES = KT + 1;
@@ -494,7 +497,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
     __syncthreads();
     stage(ncand);
     float m = -INFINITY;
-#pragma unroll 2
+#pragma unroll 4
     for (int c = 0; c < ncand; ++c) {
         const int n = ncs[c];
         const float xv = n > 0 ? fmaf(logit(c), a.sl2, lgn[c]) : -INFINITY;
@@ -502,7 +505,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
         m = fmaxf(m, xv);
     }
     float z = 0.f;
-#pragma unroll 2
+#pragma unroll 4
     for (int c = 0; c < ncand; ++c) {
         const float e = exp2f(E[c * ES + r] - m);   // 0 for empty nodes
         E[c * ES + r] = e;
@@ -562,7 +565,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
         // pass 1: every candidate's exponent u = sl2 S + log2 n - m and the
         // largest one (the candidates are independent: unrolled for overlap)
         float umax = -INFINITY;
-#pragma unroll 2
+#pragma unroll 4
         for (int c = 0; c < ncand; ++c) {
             const int n = ncs[c];
             const float u = n > 0 ? fmaf(logit(c), a.sl2, lgn[c]) - m : -INFINITY;
@@ -584,7 +587,7 @@ deep_attention_kernel(const DeepAttnArgs a) {
         }
         // pass 2: weights e' = 2^u, the corrections (A_g - A_f) n_g into Zbar
         // and Xbar
-#pragma unroll 2
+#pragma unroll 4
         for (int c = 0; c < ncand; ++c) {
             const int n = ncs[c];
             float e = 0.f;
