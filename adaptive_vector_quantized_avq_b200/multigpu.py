@@ -8,7 +8,8 @@ all-reduce of the per-rank times, so that the reported time is the slowest
 rank's.
 
 For few, long sequences the keys and queries of each (b,h) can instead be
-split along N (``sequence_sharded_forward``): every rank assigns its own keys,
+split along N (``sequence_sharded_forward``, and
+``sequence_sharded_forward_deep`` for a depth-L tree): every rank assigns its own keys,
 one SUM all-reduce of the counts and value sums makes the statistics global,
 and every rank attends its own queries. Selection depends only on the global
 statistics and on tiles, so tiles must not straddle ranks.
@@ -93,8 +94,33 @@ def sequence_sharded_forward(K, V, Q, codebook, M0: int, C: int, P: int, tile: i
         precompute = precompute or binding.precompute
         attention = attention or binding.attention
     assign, counts, vsum = precompute(K, V, codebook, M0, C)
+    _global_statistics(counts, vsum, group)
+    O, selected = attention(Q, codebook, counts, vsum, M0, C, P, tile, scale)
+    return assign, counts, vsum, O, selected
+
+
+def sequence_sharded_forward_deep(K, V, Q, codebook, M0: int, C: int, L: int, P, tile: int, scale: float,
+                                  *, precompute=None, attention=None, group=None):
+    """``sequence_sharded_forward`` over a depth-L codebook tree (the depth-L
+    calls; P: one budget per expanded level, L - 1 of them). A node's count
+    and value sum are sums over the keys whose path passes through it, so the
+    same single SUM all-reduce makes them global; the tile-level selections
+    of every level depend only on those and on the tile's own queries.
+    codebook: the full [H, Mtot, d] tree. Returns what
+    ``sequence_sharded_forward`` returns."""
+    if precompute is None or attention is None:
+        from . import binding
+        precompute = precompute or binding.precompute_deep
+        attention = attention or binding.attention_deep
+    assign, counts, vsum = precompute(K, V, codebook, M0, C, L)
+    _global_statistics(counts, vsum, group)
+    O, selected = attention(Q, codebook, counts, vsum, M0, C, L, P, tile, scale)
+    return assign, counts, vsum, O, selected
+
+
+def _global_statistics(counts, vsum, group=None) -> None:
+    """Sum the ranks' per-node counts and value sums in place (the one
+    exchange step of sequence sharding; nothing on one rank)."""
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(counts, op=dist.ReduceOp.SUM, group=group)
         dist.all_reduce(vsum, op=dist.ReduceOp.SUM, group=group)
-    O, selected = attention(Q, codebook, counts, vsum, M0, C, P, tile, scale)
-    return assign, counts, vsum, O, selected

@@ -148,3 +148,81 @@ def test_sequence_sharded_forward_equals_one_rank(oracle):
         np.testing.assert_array_equal(assign, full_pre["assign"][:, :, n0:n1])
         np.testing.assert_allclose(O, full_att["O_full"][:, :, n0:n1], rtol=1e-10, atol=1e-12)
         np.testing.assert_array_equal(sel, full_att["selected_full"][:, :, n0 // wl.tile:n1 // wl.tile])
+
+
+def _deep_oracle_calls(deep):
+    """The depth-L oracle behind the depth-L calls' signatures; selected as
+    [B, H, ntiles, sum P] (each level's expanded row ids by rank)."""
+    def pre(K, V, cb, M0, C, L):
+        r = deep.precompute(K.numpy(), V.numpy(), cb.numpy(), M0, C, L)
+        return (torch.from_numpy(r["assign"]), torch.from_numpy(r["counts"]),
+                torch.from_numpy(r["vsum"]))
+
+    def att(Q, cb, counts, vsum, M0, C, L, P, tile, scale):
+        r = deep.attention(Q.numpy(), cb.numpy(), counts.numpy(), vsum.numpy(), M0, C, L, list(P), tile, scale)
+        B, H, N, _ = Q.shape
+        ntiles = (N + tile - 1) // tile
+        sel = np.full((B * H * ntiles, sum(P)), -1, dtype=np.int64)
+        for j, levels in enumerate(r["selected"]):
+            flat = np.concatenate([np.asarray(x, dtype=np.int64) for x in levels])
+            sel[j, :flat.size] = flat
+        return torch.from_numpy(r["O_full"]), torch.from_numpy(sel.reshape(B, H, ntiles, sum(P)))
+    return pre, att
+
+
+DEEP_SHARD_WL = dict(B=1, H=2, N=640, d=8, M0=4, C=2, L=3, P=((2, 3),), tile=64, dtype="f32", seed=37,
+                     n_components=8)
+
+
+def _deep_shard_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    try:
+        from oracle import deep
+        mg.init("gloo", timeout_s=60)
+        wl = syn.small_workload(**DEEP_SHARD_WL)
+        inp = syn.generate(wl)
+        n0, n1 = mg.shard_rows(wl.N, world, rank, wl.tile)
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(inp.f64(a)[:, :, n0:n1]))
+        pre, att = _deep_oracle_calls(deep)
+        out = mg.sequence_sharded_forward_deep(t("K"), t("V"), t("Q"), torch.from_numpy(inp.f64("codebook")),
+                                               wl.M0, wl.C, wl.L, wl.P[0], wl.tile, wl.softmax_scale,
+                                               precompute=pre, attention=att)
+        dist.destroy_process_group()
+        q.put((rank, "ok", (n0, n1), [x.numpy() for x in out]))
+    except Exception as e:  # report to the parent instead of hanging it
+        q.put((rank, f"error: {e!r}", None, None))
+
+
+def test_sequence_sharded_deep_forward_equals_one_rank():
+    """Two gloo ranks, each with half of every sequence, reproduce the
+    single-rank depth-3 forward pass: global node statistics, every local
+    assignment, output row and per-level tile selection."""
+    from oracle import deep
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_deep_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    wl = syn.small_workload(**DEEP_SHARD_WL)
+    inp = syn.generate(wl)
+    pre, att = _deep_oracle_calls(deep)
+    f = lambda a: torch.from_numpy(inp.f64(a))
+    assign_f, counts_f, vsum_f = (x.numpy() for x in pre(f("K"), f("V"), f("codebook"), wl.M0, wl.C, wl.L))
+    O_f, sel_f = (x.numpy() for x in att(f("Q"), f("codebook"), torch.from_numpy(counts_f),
+                                         torch.from_numpy(vsum_f), wl.M0, wl.C, wl.L, wl.P[0], wl.tile,
+                                         wl.softmax_scale))
+    assert (assign_f >= wl.M0 + wl.M0 * wl.C).any(), "no key reached the deepest level"
+    for rank, status, (n0, n1), (assign, counts, vsum, O, sel) in res:
+        assert status == "ok", status
+        np.testing.assert_array_equal(counts, counts_f)
+        np.testing.assert_allclose(vsum, vsum_f, rtol=1e-12, atol=1e-12)
+        np.testing.assert_array_equal(assign, assign_f[:, :, n0:n1])
+        np.testing.assert_allclose(O, O_f[:, :, n0:n1], rtol=1e-10, atol=1e-12)
+        np.testing.assert_array_equal(sel, sel_f[:, :, n0 // wl.tile:n1 // wl.tile])
