@@ -604,7 +604,7 @@ def run_reference(args):
     }), flush=True)
 
 
-KERNEL_NAMES = {"precompute": ("precompute_tc_kernel", "flat_precompute_kernel", "deep_precompute_kernel"),
+KERNEL_NAMES = {"precompute": ("precompute_tc_kernel", "flat_precompute_kernel", "deep_precompute_rows_kernel"),
                 "attention": ("attention_tree_kernel", "flat_attention_kernel", "deep_attention_kernel")}
 
 

@@ -111,3 +111,16 @@ def test_traffic_hash_follows_each_path_sources(tmp_path, monkeypatch):
         f.write("\n// edit\n")
     assert bench.kernel_source_hash("attention") != tree0
     assert bench.kernel_source_hash("attention", True) == deep1
+
+
+def test_kernel_names_are_kernels_of_the_sources():
+    """Every name the ncu ingest matches is a kernel the sources define (a
+    renamed kernel would otherwise drop out of the traffic record)."""
+    import glob
+    import re
+    src = "".join(open(f).read() for f in glob.glob(os.path.join(bench.ROOT, "adaptive_vector_quantized_avq_b200",
+                                                                  "csrc", "*.cu")))
+    defined = set(re.findall(r"__global__[^;{]*?\b([a-z_0-9]+_kernel)\s*\(", src, flags=re.S))
+    for kind, names in bench.KERNEL_NAMES.items():
+        for n in names:
+            assert n in defined, (kind, n, sorted(defined))
