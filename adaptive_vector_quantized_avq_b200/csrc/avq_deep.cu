@@ -375,10 +375,10 @@ struct DeepAttnArgs {
 // per-candidate loop reads shared-memory broadcasts; without (when they would
 // not fit) it reads them from global memory, 16 bytes at a time. The
 // candidate loops are unrolled four ways (more shared-memory reads in
-// flight); at d = 64 the launch bound keeps that within the registers of
-// three CTAs per SM.
+// flight); for bf16 at d = 64 the launch bound keeps that within the
+// registers of three CTAs per SM.
 template <typename T, int D, int KT, int KC, bool ST>
-__global__ void __launch_bounds__(KT, D == 64 ? 3 : 1)
+__global__ void __launch_bounds__(KT, (D == 64 && sizeof(T) == 2) ? 3 : 1)
 deep_attention_kernel(const DeepAttnArgs a) {
     extern __shared__ float sm[];
     constexpr int ES = KT + 1;

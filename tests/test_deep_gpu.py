@@ -45,6 +45,7 @@ TREE_CASES = [
     ("L4", (4, 2, 4, 500, 64), (2, 2, 2), 128, "bf16", 1, 2, 3),
     ("L3-d128", (32, 8, 3, 4096, 128), (8, 16), 128, "bf16", 1, 2, 4),
     ("L3-f32-tile64", (8, 4, 3, 700, 64), (2, 4), 64, "f32", 1, 2, 5),
+    ("L3-f32-tile128", (16, 4, 3, 900, 64), (4, 8), 128, "f32", 1, 2, 10),
     ("L3-all", (8, 4, 3, 600, 64), (8, 32), 128, "bf16", 1, 1, 6),
     ("L3-none", (8, 4, 3, 600, 64), (0, 0), 128, "bf16", 1, 1, 7),
     ("L2", (16, 4, 2, 900, 64), (5,), 64, "bf16", 1, 2, 8),
