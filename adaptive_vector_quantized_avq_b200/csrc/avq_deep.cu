@@ -117,10 +117,10 @@ __device__ __forceinline__ float sub_bf16_hi(float k, uint32_t w) {
 // at the same time: broadcasts) and the key row is held in registers. Each
 // step is decided on fp32 squared distances (fma(t, t) over t = fl(k - c),
 // even and odd terms in two sums added at the end, whose error is bounded by
-// dist_eps); where the bound cannot
-// separate the winner from another candidate, the step is decided again on
-// exact fp64 distances (exact_sq_dist: index order, no fusion) among the
-// candidates it cannot separate, so that every decision is the exact one:
+// dist_eps); where the bound cannot separate the winner from another
+// candidate, the step is decided again on exact fp64 distances
+// (exact_sq_dist: index order, no fusion) among the candidates it cannot
+// separate, so that every decision is the exact one:
 // level 0 the nearest node (first on ties), deeper levels a child only when
 // strictly closer than the current node (first child on ties). The key's
 // own node (the deepest on its path) counts it and sums its value row
@@ -226,9 +226,8 @@ deep_precompute_rows_kernel(const T* __restrict__ K, const T* __restrict__ V, co
     for (int l = 1; l < t.L; ++l) {
         const int first = t.off[l] + local * t.C;
         // the current node first, then its children in index order; a child
-        // wins only when strictly closer
-        // (the first kCh children's distances stay in registers for the
-        // separation test)
+        // wins only when strictly closer (the first kCh children's distances
+        // stay in registers for the separation test)
         float lo = best;
         int ci = -1;
         float dch[kCh];
